@@ -1,0 +1,155 @@
+/*
+ * mla_decode.h — C ABI of the B200 (sm_100a) absorbed-MQA MLA decode library.
+ *
+ * The operation (one decode step of Multi-Head Latent Attention in its
+ * absorbed, multi-query form):
+ *
+ *   For request b, new-token index s < s_q and head h, with L_b the cached
+ *   length and L_vis = L_b - s_q + 1 + s when causal (else L_b):
+ *     z_t = softmax_scale * <q[b,s,h,0:576], row_t[0:576]>,  t < L_vis
+ *     out[b,s,h,:] = sum_t softmax(z)_t * row_t[0:512]
+ *     lse[b,h,s]   = log(sum_t exp(z_t))                      (natural log)
+ *   where row_t = kv_cache[block_table[b][t/64]][t%64][0][:].
+ *
+ *   - All heads attend directly to one shared latent cache whose rows are a
+ *     512-wide latent plus a 64-wide shared RoPE key: the full row is the key,
+ *     the latent is the value.  GQLA technical summary (gist.science, pt,
+ *     2605.15250), "Caminho MQA-Absorvido"; FlashMLA-ETAP technical summary
+ *     (gist.science, pt, 2506.01969), "Limitações" (16 heads, head dim 576).
+ *   - The kernel evaluates it in the transposed order S^T = K Q^T,
+ *     P^T = softmax(S^T) over the KV axis, O = (V^T P^T)^T, so that the long
+ *     KV axis is the MMA M dimension and heads x s_q is N.  FlashMLA-ETAP
+ *     technical summary, "Mecanismo Central" (and the arXiv abstract of
+ *     2506.01969 on fugumt.com).  The result equals the definition above up
+ *     to floating-point rounding.
+ *   - Long KV ranges are split across CTAs (split-KV); the fp32 partials are
+ *     merged by LSE weighting, which is exact: the softmax over a union of
+ *     disjoint ranges is the LSE-weighted mix of the per-range softmaxes.
+ *
+ * Conventions for every entry point:
+ *   - Data pointers are CUDA device pointers owned by the caller (e.g. from
+ *     PyTorch); the library never allocates or frees device memory, never
+ *     synchronises the device (except mla_decode_get_status, which copies one
+ *     word to the host), and enqueues work only on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream).
+ *   - Every device pointer must be 16-byte aligned and every tensor
+ *     contiguous in the layout stated.
+ *   - Return value: MLA_OK (0) or a negative MLA_ERR_* code; arguments are
+ *     checked before anything is enqueued, so an error return means nothing
+ *     was launched.  mla_decode_strerror() names a code.
+ *   - Faults the device detects while running (a block-table entry outside
+ *     [0, num_blocks), a cache length outside [0, 64*max_blocks_per_seq), a
+ *     pipeline wait that exceeded its time limit) are OR-ed as MLA_STATUS_*
+ *     bits into a status word kept in the schedule buffer; the kernels skip or
+ *     clamp the offending access instead of trapping.  The word is cleared by
+ *     mla_decode_get_schedule and read with mla_decode_get_status.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define MLA_OK 0
+#define MLA_ERR_INVALID_ARG (-1)  /* null or misaligned pointer, negative size, bad dims */
+#define MLA_ERR_UNSUPPORTED (-2)  /* page_size != 64, d_qk != 576, d_v != 512, heads*s_q > 256 */
+#define MLA_ERR_CUDA (-3)         /* a CUDA runtime/driver call or launch failed */
+#define MLA_ERR_BAD_SCHEDULE (-4) /* schedule buffer was not built for these dims */
+
+/* device status bits (mla_decode_get_status) */
+#define MLA_STATUS_BAD_BLOCK_TABLE 0x1 /* an entry was outside [0, num_blocks); page 0 was read instead */
+#define MLA_STATUS_TIMEOUT 0x2         /* a pipeline wait exceeded its limit; that CTA stopped early */
+#define MLA_STATUS_BAD_SEQLEN 0x4      /* cache_seqlens[b] outside [0, 64*max_blocks_per_seq]; clamped */
+#define MLA_STATUS_BAD_SCHEDULE 0x8    /* schedule header did not match the launch; nothing written */
+
+/* dims.flags */
+#define MLA_FLAG_NO_COMBINE 0x1 /* mla_decode_fwd does not enqueue the combine; call mla_decode_combine */
+
+typedef struct mla_decode_dims {
+    int32_t batch;              /* B >= 1 */
+    int32_t s_q;                /* new tokens per request, >= 1 (1 or 2 in the workloads) */
+    int32_t num_heads;          /* h >= 1, h * s_q <= 256 */
+    int32_t num_blocks;         /* pages in the pool */
+    int32_t max_blocks_per_seq; /* row stride of block_table */
+    int32_t page_size;          /* must be 64 */
+    int32_t d_qk;               /* must be 576 (512 latent + 64 RoPE) */
+    int32_t d_v;                /* must be 512 (the latent columns) */
+    int32_t causal;             /* 1: token s sees rows [0, L - s_q + s]; ignored when s_q == 1 */
+    int32_t num_sms;            /* persistent CTAs; 0 = the current device's SM count */
+    int32_t flags;              /* MLA_FLAG_* */
+    int32_t reserved;           /* must be 0 */
+} mla_decode_dims;
+
+/* Size in bytes of the schedule buffer for these dims (0 if dims are invalid
+ * or num_sms == 0 and no device can be queried). */
+size_t mla_decode_schedule_bytes(const mla_decode_dims* dims);
+
+/* Size in bytes of the workspace: fp32 partial outputs and LSEs of split
+ * requests (at most 2 per persistent CTA). 0 if dims are invalid. */
+size_t mla_decode_workspace_bytes(const mla_decode_dims* dims);
+
+/* Split-KV work partitioning.  Reads cache_seqlens (device, int32 [batch])
+ * and writes the persistent-CTA work plan into `schedule` (device,
+ * mla_decode_schedule_bytes(dims) bytes).  Each request x head-group costs
+ * its page count plus a fixed overhead; the total is cut into equal
+ * contiguous ranges, one per CTA, so a long request is spread over several
+ * CTAs and short ones share a CTA.  Recompute whenever cache_seqlens
+ * changes; the plan can be reused by every layer of one decode step.
+ * Clears the device status word. */
+int mla_decode_get_schedule(const mla_decode_dims* dims, const int32_t* cache_seqlens,
+                            void* schedule, void* stream);
+
+/* The same plan computed on the host from host arrays (for inspection and
+ * tests); `schedule_host` is host memory of mla_decode_schedule_bytes(dims)
+ * bytes.  dims->num_sms must be > 0.  No CUDA call is made. */
+int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* cache_seqlens_host,
+                                 void* schedule_host);
+
+/* Decode attention.
+ *   q            bf16 [batch][s_q][num_heads][576]
+ *   kv_cache     bf16 [num_blocks][64][1][576]   (page pool; 73,728 B per page)
+ *   block_table  int32 [batch][max_blocks_per_seq]: page ids; only the first
+ *                ceil(L_b / 64) entries of row b are read
+ *   cache_seqlens int32 [batch]: L_b, the cached length including the s_q new tokens
+ *   softmax_scale scale applied to q.k (e.g. 192^-0.5)
+ *   out          bf16 [batch][s_q][num_heads][512]
+ *   lse          fp32 [batch][num_heads][s_q]  (natural log; -inf if nothing is visible)
+ *   schedule     from mla_decode_get_schedule with the same dims and lengths
+ *   workspace    mla_decode_workspace_bytes(dims) bytes, no initialisation needed
+ * Enqueues the persistent decode kernel and then (unless MLA_FLAG_NO_COMBINE)
+ * the combine kernel on `stream`.  A request whose visible range is empty
+ * gets out = 0 and lse = -inf. */
+int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* workspace,
+                   const void* q, const void* kv_cache, const int32_t* block_table,
+                   const int32_t* cache_seqlens, float softmax_scale, void* out, float* lse,
+                   void* stream);
+
+/* LSE-weighted merge of the split partials left in `workspace` by
+ * mla_decode_fwd: L* = log sum_i exp(lse_i), out = sum_i exp(lse_i - L*) O_i.
+ * Also writes out = 0, lse = -inf for empty requests.  Requests that were not
+ * split were already written by mla_decode_fwd and are not touched. */
+int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const void* workspace,
+                       void* out, float* lse, void* stream);
+
+/* Copies the device status word (OR of MLA_STATUS_* bits since the last
+ * mla_decode_get_schedule) to *host_status.  Synchronous: waits for the copy
+ * on the legacy default stream, so call it after the work it should cover has
+ * finished (e.g. after synchronising the stream that ran it). */
+int mla_decode_get_status(const void* schedule, int32_t* host_status);
+
+/* Static text for an MLA_* return code. */
+const char* mla_decode_strerror(int code);
+
+/* Library ABI version (increments on any change of these declarations). */
+int mla_decode_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

@@ -1,0 +1,236 @@
+"""Python binding of the C ABI in include/mla_decode.h (ctypes).
+
+Argument marshalling only: every step of the decode runs in the CUDA kernels
+of libmla_decode.so.  PyTorch supplies device memory and the stream.  There is
+no fallback: if the library is missing or the device is not an sm_100 part,
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from . import _build
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = -1
+MLA_ERR_UNSUPPORTED = -2
+MLA_ERR_CUDA = -3
+MLA_ERR_BAD_SCHEDULE = -4
+
+MLA_STATUS_BAD_BLOCK_TABLE = 0x1
+MLA_STATUS_TIMEOUT = 0x2
+MLA_STATUS_BAD_SEQLEN = 0x4
+MLA_STATUS_BAD_SCHEDULE = 0x8
+
+MLA_FLAG_NO_COMBINE = 0x1
+
+PAGE_SIZE = 64
+D_QK = 576
+D_V = 512
+
+EXPORTED = (
+    "mla_decode_schedule_bytes",
+    "mla_decode_workspace_bytes",
+    "mla_decode_get_schedule",
+    "mla_decode_get_schedule_host",
+    "mla_decode_fwd",
+    "mla_decode_combine",
+    "mla_decode_get_status",
+    "mla_decode_strerror",
+    "mla_decode_version",
+)
+
+
+class MlaDecodeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (where, mla_decode_strerror(code), code))
+
+
+class mla_decode_dims(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "batch", "s_q", "num_heads", "num_blocks", "max_blocks_per_seq", "page_size",
+        "d_qk", "d_v", "causal", "num_sms", "flags", "reserved")]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmla_decode.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_build.LIB):
+            raise RuntimeError("CUDA library %s is not built; run __graft_entry__.build() "
+                               "(nvcc, sm_100a)" % _build.LIB)
+        L = ctypes.CDLL(_build.LIB)
+        P = ctypes.POINTER(mla_decode_dims)
+        vp = ctypes.c_void_p
+        L.mla_decode_schedule_bytes.restype = ctypes.c_size_t
+        L.mla_decode_schedule_bytes.argtypes = [P]
+        L.mla_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.mla_decode_workspace_bytes.argtypes = [P]
+        L.mla_decode_get_schedule.restype = ctypes.c_int
+        L.mla_decode_get_schedule.argtypes = [P, vp, vp, vp]
+        L.mla_decode_get_schedule_host.restype = ctypes.c_int
+        L.mla_decode_get_schedule_host.argtypes = [P, vp, vp]
+        L.mla_decode_fwd.restype = ctypes.c_int
+        L.mla_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+        L.mla_decode_combine.restype = ctypes.c_int
+        L.mla_decode_combine.argtypes = [P, vp, vp, vp, vp, vp]
+        L.mla_decode_get_status.restype = ctypes.c_int
+        L.mla_decode_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.mla_decode_strerror.restype = ctypes.c_char_p
+        L.mla_decode_strerror.argtypes = [ctypes.c_int]
+        L.mla_decode_version.restype = ctypes.c_int
+        L.mla_decode_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def make_dims(batch: int, s_q: int, num_heads: int, num_blocks: int, max_blocks_per_seq: int,
+              causal: bool = False, num_sms: int = 0, flags: int = 0) -> mla_decode_dims:
+    return mla_decode_dims(int(batch), int(s_q), int(num_heads), int(num_blocks),
+                           int(max_blocks_per_seq), PAGE_SIZE, D_QK, D_V, int(bool(causal)),
+                           int(num_sms), int(flags), 0)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MLA_OK:
+        raise MlaDecodeError(rc, where)
+
+
+def mla_decode_strerror(code: int) -> str:
+    return lib().mla_decode_strerror(int(code)).decode()
+
+
+def mla_decode_version() -> int:
+    return int(lib().mla_decode_version())
+
+
+def mla_decode_schedule_bytes(dims: mla_decode_dims) -> int:
+    return int(lib().mla_decode_schedule_bytes(ctypes.byref(dims)))
+
+
+def mla_decode_workspace_bytes(dims: mla_decode_dims) -> int:
+    return int(lib().mla_decode_workspace_bytes(ctypes.byref(dims)))
+
+
+def mla_decode_get_schedule(dims, cache_seqlens: torch.Tensor, schedule: torch.Tensor, stream=None) -> None:
+    _check(lib().mla_decode_get_schedule(ctypes.byref(dims), _ptr(cache_seqlens), _ptr(schedule),
+                                         _stream(stream)), "mla_decode_get_schedule")
+
+
+def mla_decode_get_schedule_host(dims, cache_seqlens, schedule) -> None:
+    """Host version; ``cache_seqlens`` (int32) and ``schedule`` are CPU tensors."""
+    _check(lib().mla_decode_get_schedule_host(ctypes.byref(dims), _ptr(cache_seqlens), _ptr(schedule)),
+           "mla_decode_get_schedule_host")
+
+
+def mla_decode_fwd(dims, schedule, workspace, q, kv_cache, block_table, cache_seqlens,
+                   softmax_scale: float, out, lse, stream=None) -> None:
+    _check(lib().mla_decode_fwd(ctypes.byref(dims), _ptr(schedule), _ptr(workspace), _ptr(q),
+                                _ptr(kv_cache), _ptr(block_table), _ptr(cache_seqlens),
+                                float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_decode_fwd")
+
+
+def mla_decode_combine(dims, schedule, workspace, out, lse, stream=None) -> None:
+    _check(lib().mla_decode_combine(ctypes.byref(dims), _ptr(schedule), _ptr(workspace), _ptr(out),
+                                    _ptr(lse), _stream(stream)), "mla_decode_combine")
+
+
+def mla_decode_get_status(schedule: torch.Tensor) -> int:
+    v = ctypes.c_int32(0)
+    _check(lib().mla_decode_get_status(_ptr(schedule), ctypes.byref(v)), "mla_decode_get_status")
+    return int(v.value)
+
+
+def _require(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+class MlaDecoder:
+    """Owns the schedule and workspace buffers for one shape of decode batch.
+
+    ``plan(cache_seqlens)`` builds the split-KV schedule (once per decode step);
+    ``__call__`` runs the decode kernel + combine and returns (out, lse).
+    """
+
+    def __init__(self, batch: int, s_q: int, num_heads: int, num_blocks: int,
+                 max_blocks_per_seq: int, causal: bool = False, num_sms: int = 0,
+                 device: Optional[torch.device] = None):
+        self.device = torch.device(device or "cuda")
+        if num_sms == 0:
+            num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        self.dims = make_dims(batch, s_q, num_heads, num_blocks, max_blocks_per_seq, causal, num_sms)
+        sb = mla_decode_schedule_bytes(self.dims)
+        wb = mla_decode_workspace_bytes(self.dims)
+        if sb == 0 or wb == 0:
+            raise MlaDecodeError(MLA_ERR_INVALID_ARG, "MlaDecoder dims")
+        self.schedule = torch.empty(sb, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.empty(wb, dtype=torch.uint8, device=self.device)
+        self.out = torch.empty(batch, s_q, num_heads, D_V, dtype=torch.bfloat16, device=self.device)
+        self.lse = torch.empty(batch, num_heads, s_q, dtype=torch.float32, device=self.device)
+
+    def check_inputs(self, q, kv_cache, block_table, cache_seqlens) -> None:
+        d = self.dims
+        _require(q.dtype == torch.bfloat16 and q.is_contiguous() and
+                 tuple(q.shape) == (d.batch, d.s_q, d.num_heads, D_QK), "q must be bf16 [B, s_q, h, 576]")
+        _require(kv_cache.dtype == torch.bfloat16 and kv_cache.is_contiguous() and
+                 kv_cache.shape[0] == d.num_blocks and kv_cache.shape[1] == PAGE_SIZE and
+                 kv_cache.shape[-1] == D_QK and kv_cache.numel() == d.num_blocks * PAGE_SIZE * D_QK,
+                 "kv_cache must be bf16 [num_blocks, 64, 1, 576]")
+        _require(block_table.dtype == torch.int32 and block_table.is_contiguous() and
+                 tuple(block_table.shape) == (d.batch, d.max_blocks_per_seq),
+                 "block_table must be int32 [B, max_blocks_per_seq]")
+        _require(cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and
+                 tuple(cache_seqlens.shape) == (d.batch,), "cache_seqlens must be int32 [B]")
+        for t in (q, kv_cache, block_table, cache_seqlens):
+            _require(t.device == self.out.device, "all tensors must be on %s" % self.out.device)
+
+    def plan(self, cache_seqlens: torch.Tensor, stream=None) -> None:
+        mla_decode_get_schedule(self.dims, cache_seqlens, self.schedule, stream)
+
+    def __call__(self, q, kv_cache, block_table, cache_seqlens, softmax_scale: float,
+                 stream=None, check: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+        if check:
+            self.check_inputs(q, kv_cache, block_table, cache_seqlens)
+        mla_decode_fwd(self.dims, self.schedule, self.workspace, q, kv_cache, block_table,
+                       cache_seqlens, softmax_scale, self.out, self.lse, stream)
+        return self.out, self.lse
+
+    def status(self) -> int:
+        return mla_decode_get_status(self.schedule)
+
+
+def mla_decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor,
+               cache_seqlens: torch.Tensor, softmax_scale: float, causal: bool = False,
+               num_sms: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One-shot convenience: plan + decode on the current stream; returns (out, lse)."""
+    B, s_q, h, _ = q.shape
+    dec = MlaDecoder(B, s_q, h, kv_cache.shape[0], block_table.shape[1], causal, num_sms, q.device)
+    dec.plan(cache_seqlens)
+    out, lse = dec(q, kv_cache, block_table, cache_seqlens, softmax_scale)
+    return out.clone(), lse.clone()

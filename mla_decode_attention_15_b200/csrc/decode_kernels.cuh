@@ -1,0 +1,814 @@
+// sm_100a kernels of absorbed-MQA MLA decode in the transposed ("ETAP") order.
+//
+// Method (FlashMLA-ETAP technical summary, gist.science pt 2506.01969,
+// "Mecanismo Central"): instead of S = Q K^T, softmax over keys, O = P V,
+// compute S^T = K Q^T, P^T = softmax(S^T) along the KV axis and
+// O = (V^T P^T)^T, so the long KV axis is the MMA M dimension and the few
+// query columns (heads x new tokens) are N.  The cache is the absorbed-MQA
+// latent cache of the GQLA summary (gist.science pt 2605.15250, "Caminho
+// MQA-Absorvido"): one 576-wide row per token, key = whole row, value = the
+// first 512 columns.  "Detalhes de Implementação" of the FlashMLA-ETAP summary
+// describes a producer/consumer split inside one CTA on Hopper; here the roles
+// are re-cut for Blackwell:
+//
+//   warp 0        TMA producer: Q of the work item, then every 64-token page
+//                 gathered through the block table (9 boxes of 64x64 bf16,
+//                 128-byte swizzle) into a 2-stage ring of 72 KB stages.
+//   warp 1        one thread issues tcgen05.mma:
+//                   GEMM1  S^T[64 x N]  = K[64 x 576] . Q^T        (M=64, K-major A and B)
+//                   GEMM2  O^T[512 x N] += V^T[512 x 64] . P^T     (4 x M=128, MN-major A and B)
+//                 accumulators live in TMEM; V^T is the same shared-memory page
+//                 read through a second (MN-major) descriptor.
+//   warps 2..5    softmax over the KV axis (one TMEM lane = one token), lazy
+//                 rescale of O^T in TMEM, P^T to shared memory as bf16, and the
+//                 epilogue (O = O^T / l transposed back, LSE), either final or
+//                 as an fp32 partial of a split request.
+//
+// Every wait on an mbarrier is bounded: after kWaitLimitNs the waiting role
+// raises MLA_STATUS_TIMEOUT and a CTA-wide abort flag, all roles leave their
+// loops, in-flight copies and MMAs are drained (again with a limit) and TMEM
+// is released before the CTA exits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "schedule.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+
+constexpr uint32_t kFullMask = 0xffffffffu;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr int kFwdThreads = 192;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the running max grows by > 2^8
+constexpr float kLn2 = 0.693147180559945309f;
+
+struct FwdParams {
+    const int32_t* sched;
+    const int32_t* block_table;
+    const int32_t* seqlens;
+    __nv_bfloat16* out;
+    float* lse;
+    float* opart;  // [slots][NG][512]
+    float* lpart;  // [slots][NG]
+    int32_t* status;
+    int s_q, heads, N, num_blocks, max_blocks, causal;
+    int G, BG, Hg, slots_cap;
+    float scale_log2;  // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+    const int32_t* sched;
+    const float* opart;
+    const float* lpart;
+    __nv_bfloat16* out;
+    float* lse;
+    int32_t* status;
+    int s_q, heads, N, NG, Hg, G, BG, slots_cap;
+};
+
+// ------------------------------------------------------------------ layout
+template <int NG>
+struct FwdSmem {
+    static constexpr int kStages = 2;
+    static constexpr int kBoxCols = 64;
+    static constexpr int kBoxBytes = kPage * kBoxCols * 2;    // 8 KB: 64 tokens x 64 cols
+    static constexpr int kBoxes = kDqk / kBoxCols;            // 9
+    static constexpr int kStageBytes = kBoxes * kBoxBytes;    // 72 KB: one page
+    static constexpr int kQBoxBytes = NG * 128;               // NG rows x 64 cols
+    static constexpr int kQBytes = kBoxes * kQBoxBytes;
+    static constexpr int kPBytes = kPage * NG * 2;            // P^T of one page, bf16
+    static constexpr int kKvOff = 0;
+    static constexpr int kQOff = kKvOff + kStages * kStageBytes;
+    static constexpr int kPOff = kQOff + kQBytes;
+    static constexpr int kRedOff = kPOff + 2 * kPBytes;       // float [2][NG][4] page maxima
+    static constexpr int kSumOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]   row sums
+    static constexpr int kBarOff = kSumOff + NG * 4 * 4;
+    static constexpr int kNumBars = 20;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
+    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KB
+    static constexpr int kTmemCols = NG == 16 ? 128 : 256;    // 2 S^T buffers + O^T (4 chunks)
+    static constexpr int kSCol = 0;                           // S^T buffer i at column i*NG
+    static constexpr int kOCol = 2 * NG;                      // O^T chunk c at column kOCol + c*NG
+    static_assert(6 * NG <= kTmemCols, "TMEM budget");
+    static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0, "swizzle atoms need 1 KB alignment");
+    static_assert(kBytes <= 227 * 1024, "shared memory budget");
+};
+
+enum Bar {
+    kKvFull0 = 0, kKvFull1, kKvEmpty0, kKvEmpty1, kQFull, kQEmpty,
+    kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
+    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kBarCount
+};
+
+// ------------------------------------------------------------------ waits
+struct Ctl {
+    volatile int* abort_flag;
+    int32_t* status;
+};
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*c.abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *c.abort_flag = 1;
+            atomicOr(c.status, MLA_STATUS_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// All 32 lanes wait; the verdict is made warp-uniform so that the warp keeps
+// executing .sync.aligned instructions together.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& c) {
+    const bool ok = wait_bounded(bar, parity, c);
+    return __all_sync(kFullMask, ok);
+}
+
+// Teardown wait: ignores the abort flag, bounded by time only.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ work walk
+struct Item {
+    int bg, b, g, p0, p1, P, L, slot;
+    bool unsplit;
+};
+
+struct WorkIter {
+    int bg, begin_bg, begin_page, end_bg, end_page, first_split;
+
+    __device__ void init(const int32_t* meta) {
+        begin_bg = __ldg(meta + kMetaBeginBg);
+        begin_page = __ldg(meta + kMetaBeginPage);
+        end_bg = __ldg(meta + kMetaEndBg);
+        end_page = __ldg(meta + kMetaEndPage);
+        first_split = __ldg(meta + kMetaFirstSplit);
+        bg = begin_bg;
+    }
+
+    __device__ bool next(const FwdParams& p, const int32_t* bginfo, Item& it) {
+        while (bg <= end_bg && bg < p.BG) {
+            const int cur = bg++;
+            const int b = cur / p.Hg;
+            const int L = clamp_seqlen(__ldg(p.seqlens + b), p.max_blocks);
+            const int P = pages_of(L);
+            const int p0 = (cur == begin_bg) ? begin_page : 0;
+            int p1 = (cur == end_bg) ? end_page : P;
+            if (p1 > P) p1 = P;
+            if (p0 >= p1) continue;
+            it.bg = cur;
+            it.b = b;
+            it.g = cur - b * p.Hg;
+            it.p0 = p0;
+            it.p1 = p1;
+            it.P = P;
+            it.L = L;
+            it.unsplit = (p0 == 0 && p1 == P);
+            it.slot = -1;
+            if (!it.unsplit) {
+                const int s = __ldg(bginfo + kBgWords * cur) + ((cur == begin_bg) ? first_split : 0);
+                it.slot = (s >= 0 && s < p.slots_cap) ? s : -1;
+            }
+            return true;
+        }
+        return false;
+    }
+};
+
+// ------------------------------------------------------------------ helpers
+// Transpose-reduce across the warp: each step every lane keeps half of its
+// columns and folds in its partner's copy of them.  After it, the lane holds
+// the reduction over all 32 lanes of column (lane >> (5 - log2 W)).
+template <int W, int OFF, bool kMax>
+struct ColReduce {
+    __device__ __forceinline__ static float run(float* v, int lane) {
+        constexpr int H = W / 2;
+        const bool upper = (lane & OFF) != 0;
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            const float send = upper ? v[i] : v[i + H];
+            const float keep = upper ? v[i + H] : v[i];
+            const float got = __shfl_xor_sync(kFullMask, send, OFF);
+            v[i] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+        return ColReduce<H, OFF / 2, kMax>::run(v, lane);
+    }
+};
+template <int OFF, bool kMax>
+struct ColReduce<1, OFF, kMax> {
+    __device__ __forceinline__ static float run(float* v, int) {
+        float x = v[0];
+#pragma unroll
+        for (int o = OFF; o >= 1; o >>= 1) {
+            const float got = __shfl_xor_sync(kFullMask, x, o);
+            x = kMax ? fmaxf(x, got) : x + got;
+        }
+        return x;
+    }
+};
+
+template <int NG>
+__device__ __forceinline__ int reduced_col(int lane) {
+    return NG == 16 ? (lane >> 1) : lane;
+}
+template <int NG>
+__device__ __forceinline__ bool reduced_writer(int lane) {
+    return NG == 32 || (lane & 1) == 0;
+}
+
+template <int NG>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&v)[NG]) {
+#pragma unroll
+    for (int c = 0; c < NG; c += 16) {
+        float t[16];
+        tmem_ld_x16(taddr + c, t);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[c + i] = t[i];
+    }
+}
+template <int NG>
+__device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const float (&v)[NG]) {
+#pragma unroll
+    for (int c = 0; c < NG; c += 16) {
+        float t[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) t[i] = v[c + i];
+        tmem_st_x16(taddr + c, t);
+    }
+}
+
+// ------------------------------------------------------------------ roles
+template <int NG>
+__device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map,
+                             const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                             uint8_t* smem, const Ctl& ctl) {
+    using L = FwdSmem<NG>;
+    const uint32_t kv_s = smem_addr(smem + L::kKvOff);
+    const uint32_t q_s = smem_addr(smem + L::kQOff);
+    const uint32_t bar0 = smem_addr(smem + L::kBarOff);
+    const uint64_t policy = p.Hg > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
+    WorkIter it;
+    it.init(meta);
+    Item item;
+    uint32_t kv_it = 0, q_it = 0;
+    bool ok = true;
+    while (ok && it.next(p, bginfo, item)) {
+        ok = wait_bounded(bar0 + 8 * kQEmpty, (q_it & 1) ^ 1, ctl);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar0 + 8 * kQFull, L::kQBytes);
+        const int row0 = item.b * p.N + item.g * NG;
+#pragma unroll 1
+        for (int c = 0; c < L::kBoxes; ++c)
+            tma_load_2d(q_s + c * L::kQBoxBytes, q_map, bar0 + 8 * kQFull, c * L::kBoxCols, row0);
+        ++q_it;
+        const int32_t* bt = p.block_table + (size_t)item.b * p.max_blocks;
+        for (int j = item.p0; j < item.p1; ++j) {
+            const int st = kv_it & 1;
+            ok = wait_bounded(bar0 + 8 * (kKvEmpty0 + st), ((kv_it >> 1) & 1) ^ 1, ctl);
+            if (!ok) break;
+            int phys = __ldg(bt + j);
+            if ((unsigned)phys >= (unsigned)p.num_blocks) {
+                atomicOr(p.status, MLA_STATUS_BAD_BLOCK_TABLE);
+                phys = 0;
+            }
+            const uint32_t full = bar0 + 8 * (kKvFull0 + st);
+            mbar_arrive_expect_tx(full, L::kStageBytes);
+            const uint32_t dst = kv_s + st * L::kStageBytes;
+#pragma unroll
+            for (int c = 0; c < L::kBoxes; ++c)
+                tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, c * L::kBoxCols, 0, phys, policy);
+            ++kv_it;
+        }
+    }
+    if (!ok) {
+        // Let the copies already issued land before the CTA exits.
+        for (int st = 0; st < 2; ++st) {
+            const uint32_t n = (kv_it + 1 - st) / 2;
+            if (n > 0) wait_drain(bar0 + 8 * (kKvFull0 + st), (n - 1) & 1);
+        }
+        if (q_it > 0) wait_drain(bar0 + 8 * kQFull, (q_it - 1) & 1);
+    }
+}
+
+template <int NG>
+__device__ void run_mma(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                        uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
+    using L = FwdSmem<NG>;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(64, NG, 0, 0);   // S^T = K . Q^T
+    constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);  // O^T += V^T . P^T
+    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : kSwizzle64;
+    const uint32_t kv_s = smem_addr(smem + L::kKvOff);
+    const uint32_t q_s = smem_addr(smem + L::kQOff);
+    const uint32_t p_s = smem_addr(smem + L::kPOff);
+    const uint32_t bar0 = smem_addr(smem + L::kBarOff);
+    WorkIter it;
+    it.init(meta);
+    Item item;
+    uint32_t kv_it = 0, s_it = 0, q_it = 0, item_it = 0;
+    bool ok = true, issued = false;
+
+    // GEMM2 of one page: reads the V columns of stage `st` (MN-major: d_v is
+    // contiguous within a token row; 64 d_v per swizzle atom, next atom = next
+    // box, 8-token groups 1 KB apart) and P^T buffer (sidx & 1) (MN-major:
+    // NG columns contiguous per token row).
+    auto gemm2 = [&](int st, uint32_t sidx, bool first) -> bool {
+        const int pb = sidx & 1;
+        if (!wait_bounded(bar0 + 8 * (kPFull0 + pb), (sidx >> 1) & 1, ctl)) return false;
+        if (first && !wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t a0 = kv_s + st * L::kStageBytes;
+        const uint32_t b0 = p_s + pb * L::kPBytes;
+#pragma unroll
+        for (int ch = 0; ch < kDv / 128; ++ch) {
+            const uint32_t d = tmem + L::kOCol + ch * NG;
+#pragma unroll
+            for (int k = 0; k < kPage / 16; ++k) {
+                const uint64_t a = smem_desc(a0 + (2 * ch) * L::kBoxBytes + k * 2048, L::kBoxBytes, 1024,
+                                             kSwizzle128);
+                const uint64_t b = smem_desc(b0 + k * 16 * NG * 2, L::kPBytes, 8 * NG * 2, kPSwizzle);
+                umma_f16(d, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
+            }
+        }
+        umma_commit(bar0 + 8 * (kKvEmpty0 + st));
+        umma_commit(bar0 + 8 * (kPEmpty0 + pb));
+        return true;
+    };
+
+    while (ok && it.next(p, bginfo, item)) {
+        ok = wait_bounded(bar0 + 8 * kQFull, q_it & 1, ctl);
+        if (!ok) break;
+        const int npages = item.p1 - item.p0;
+        int pend_st = -1;
+        uint32_t pend_s = 0;
+        bool pend_first = false;
+        for (int jj = 0; jj < npages; ++jj) {
+            const int st = kv_it & 1;
+            ok = wait_bounded(bar0 + 8 * (kKvFull0 + st), (kv_it >> 1) & 1, ctl);
+            if (!ok) break;
+            const int sb = s_it & 1;
+            ok = wait_bounded(bar0 + 8 * (kSEmpty0 + sb), ((s_it >> 1) & 1) ^ 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            // GEMM1: K-major A (64 token rows of 128 B per box, 8-row groups 1 KB
+            // apart) and K-major B (Q^T rows); the 16-wide k-step advances 32 B
+            // inside the 128-byte swizzle atom.
+            const uint32_t d = tmem + L::kSCol + sb * NG;
+            const uint32_t a0 = kv_s + st * L::kStageBytes;
+#pragma unroll 1
+            for (int c = 0; c < L::kBoxes; ++c) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t a = smem_desc(a0 + c * L::kBoxBytes + k * 32, 16, 1024, kSwizzle128);
+                    const uint64_t b = smem_desc(q_s + c * L::kQBoxBytes + k * 32, 16, 1024, kSwizzle128);
+                    umma_f16(d, a, b, kIdescS, (c | k) ? 1u : 0u);
+                }
+            }
+            issued = true;
+            umma_commit(bar0 + 8 * (kSFull0 + sb));
+            if (jj == npages - 1) umma_commit(bar0 + 8 * kQEmpty);
+            if (pend_st >= 0) {
+                ok = gemm2(pend_st, pend_s, pend_first);
+                if (!ok) break;
+            }
+            pend_st = st;
+            pend_s = s_it;
+            pend_first = (jj == 0);
+            ++kv_it;
+            ++s_it;
+        }
+        if (!ok) break;
+        ok = gemm2(pend_st, pend_s, pend_first);
+        if (!ok) break;
+        ++q_it;
+        ++item_it;
+    }
+    if (issued) {
+        umma_commit(bar0 + 8 * kMmaDone);
+        wait_drain(bar0 + 8 * kMmaDone, 0);
+    }
+}
+
+template <int NG>
+__device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                            uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
+    using L = FwdSmem<NG>;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
+    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
+    const int gt = threadIdx.x - 64;                      // 0..127 within the softmax group
+    const uint32_t bar0 = smem_addr(smem + L::kBarOff);
+    float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+    float* sred = reinterpret_cast<float*>(smem + L::kSumOff);
+    uint8_t* pbuf = smem + L::kPOff;
+    // In an M=64 accumulator, token row m of S^T sits in TMEM lane 32*(m/16) + m%16:
+    // lanes 0..15 of each quadrant carry 16 tokens of the page.
+    const bool row_ok = lane < 16;
+    const int row = 16 * wq + lane;
+    constexpr int kChunks = NG * 2 / 16;  // 16-byte chunks per P^T row
+
+    WorkIter it;
+    it.init(meta);
+    Item item;
+    uint32_t s_it = 0, item_it = 0;
+    bool ok = true;
+    while (ok && it.next(p, bginfo, item)) {
+        int lvis[NG];
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+            const int gc = item.g * NG + n;
+            int v = 0;
+            if (gc < p.N) {
+                const int s = gc / p.heads;
+                v = (p.causal && p.s_q > 1) ? item.L - p.s_q + 1 + s : item.L;
+            }
+            lvis[n] = v;
+        }
+        float m_run[NG], l_run[NG];
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+            m_run[n] = -INFINITY;
+            l_run[n] = 0.f;
+        }
+        for (int j = item.p0; j < item.p1; ++j) {
+            const int sb = s_it & 1;
+            ok = wait_warp(bar0 + 8 * (kSFull0 + sb), (s_it >> 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            float x[NG];
+            tmem_load_cols<NG>(tmem + lane_base + L::kSCol + sb * NG, x);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(bar0 + 8 * (kSEmpty0 + sb));
+
+            const int t = j * kPage + row;
+#pragma unroll
+            for (int n = 0; n < NG; ++n) x[n] = (row_ok && t < lvis[n]) ? x[n] * p.scale_log2 : -INFINITY;
+
+            // Column maxima of this page: warp transpose-reduce, then the four
+            // warps meet through shared memory.
+            float xr[NG];
+#pragma unroll
+            for (int n = 0; n < NG; ++n) xr[n] = x[n];
+            const float wmax = ColReduce<NG, 16, true>::run(xr, lane);
+            float* rb = red + (s_it & 1) * NG * 4;
+            if (reduced_writer<NG>(lane)) rb[reduced_col<NG>(lane) * 4 + wq] = wmax;
+            mbar_arrive(bar0 + 8 * (kRedFull0 + (s_it & 1)));
+            ok = wait_warp(bar0 + 8 * (kRedFull0 + (s_it & 1)), (s_it >> 1) & 1, ctl);
+            if (!ok) break;
+
+            float alpha[NG];
+            bool rescale = false;
+#pragma unroll
+            for (int n = 0; n < NG; ++n) {
+                const float4 r4 = *reinterpret_cast<const float4*>(rb + n * 4);
+                const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+                const float mnew = fmaxf(m_run[n], pmax);
+                if (mnew > m_run[n] + kRescaleLog2) {
+                    alpha[n] = ex2_approx(m_run[n] - mnew);
+                    m_run[n] = mnew;
+                    rescale = true;
+                } else {
+                    alpha[n] = 1.f;
+                }
+            }
+            // P = 2^(x - m): GEMM2 multiplies its bf16 rounding; the row sums
+            // (and so the LSE) accumulate the fp32 values.
+            uint32_t packed[NG / 2];
+#pragma unroll
+            for (int n = 0; n < NG; n += 2) {
+                const float e0 = (x[n] == -INFINITY) ? 0.f : ex2_approx(x[n] - m_run[n]);
+                const float e1 = (x[n + 1] == -INFINITY) ? 0.f : ex2_approx(x[n + 1] - m_run[n + 1]);
+                l_run[n] = l_run[n] * alpha[n] + e0;
+                l_run[n + 1] = l_run[n + 1] * alpha[n + 1] + e1;
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+                packed[n / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            const int pb = s_it & 1;
+            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
+            if (!ok) break;
+            if (row_ok) {
+                // P^T row of this token, MN-major with a (2*NG)-byte swizzle span:
+                // 16-byte chunk c of row r lands at chunk c ^ ((r*2*NG >> 7) & (kChunks-1)).
+                uint8_t* rowp = pbuf + pb * L::kPBytes + row * (NG * 2);
+                const int swz = ((row * NG * 2) >> 7) & (kChunks - 1);
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    *reinterpret_cast<uint4*>(rowp + ((c ^ swz) * 16)) =
+                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            if (rescale && j > item.p0) {
+                // O^T already holds earlier pages: wait for the previous GEMM2,
+                // then scale each column by its alpha in place.
+                const uint32_t prev = s_it - 1;
+                ok = wait_warp(bar0 + 8 * (kPEmpty0 + (prev & 1)), (prev >> 1) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int ch = 0; ch < kDv / 128; ++ch) {
+                    float o[NG];
+                    const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
+                    tmem_load_cols<NG>(ta, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int n = 0; n < NG; ++n) o[n] *= alpha[n];
+                    tmem_store_cols<NG>(ta, o);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(bar0 + 8 * (kPFull0 + pb));
+            ++s_it;
+        }
+        if (!ok) break;
+
+        // ---- epilogue: wait for the last GEMM2, reduce l over the tokens ----
+        const uint32_t last = s_it - 1;
+        ok = wait_warp(bar0 + 8 * (kPEmpty0 + (last & 1)), (last >> 1) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        float lr[NG];
+#pragma unroll
+        for (int n = 0; n < NG; ++n) lr[n] = l_run[n];
+        const float wsum = ColReduce<NG, 16, false>::run(lr, lane);
+        if (reduced_writer<NG>(lane)) sred[reduced_col<NG>(lane) * 4 + wq] = wsum;
+        mbar_arrive(bar0 + 8 * kSumFull);
+        ok = wait_warp(bar0 + 8 * kSumFull, item_it & 1, ctl);
+        if (!ok) break;
+        float lsum[NG], inv[NG];
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sred + n * 4);
+            lsum[n] = (s4.x + s4.y) + (s4.z + s4.w);
+            inv[n] = lsum[n] > 0.f ? 1.f / lsum[n] : 0.f;
+        }
+#pragma unroll 1
+        for (int ch = 0; ch < kDv / 128; ++ch) {
+            float o[NG];
+            tmem_load_cols<NG>(tmem + lane_base + L::kOCol + ch * NG, o);
+            tmem_ld_wait();
+            const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
+#pragma unroll
+            for (int n = 0; n < NG; ++n) {
+                const int gc = item.g * NG + n;
+                if (gc < p.N) {
+                    const float v = o[n] * inv[n];
+                    if (item.unsplit) {
+                        const int s = gc / p.heads;
+                        const int head = gc - s * p.heads;
+                        p.out[(((size_t)item.b * p.s_q + s) * p.heads + head) * kDv + d] =
+                            __float2bfloat16_rn(v);
+                    } else if (item.slot >= 0) {
+                        p.opart[((size_t)item.slot * NG + n) * kDv + d] = v;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+            const int gc = item.g * NG + n;
+            if (gt == n && gc < p.N) {
+                const float lse2 = lsum[n] > 0.f ? m_run[n] + log2f(lsum[n]) : -INFINITY;
+                const float lse = lse2 * kLn2;
+                if (item.unsplit) {
+                    const int s = gc / p.heads;
+                    const int head = gc - s * p.heads;
+                    p.lse[((size_t)item.b * p.heads + head) * p.s_q + s] = lse;
+                } else if (item.slot >= 0) {
+                    p.lpart[(size_t)item.slot * NG + n] = lse;
+                }
+            }
+        }
+        if (!item.unsplit && item.slot < 0 && gt == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        tc_fence_before();
+        mbar_arrive(bar0 + 8 * kOEmpty);
+        ++item_it;
+    }
+}
+
+// ------------------------------------------------------------------ kernels
+template <int NG>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    mla_decode_fwd_kernel(const __grid_constant__ CUtensorMap kv_map,
+                          const __grid_constant__ CUtensorMap q_map, const FwdParams p) {
+    using L = FwdSmem<NG>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int32_t* hdr = p.sched;
+    if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
+        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG) {
+        if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        return;
+    }
+    const int32_t* meta = hdr + kHdrWords + (size_t)blockIdx.x * kMetaWords;
+    const int32_t* bginfo = hdr + bg_offset_words(p.G);
+    const uint32_t bar0 = smem_addr(smem + L::kBarOff);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kBarCount; ++i) {
+            uint32_t count = 1;
+            if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
+                i == kRedFull0 || i == kRedFull1 || i == kSumFull)
+                count = 128;
+            mbar_init(bar0 + 8 * i, count);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Ctl ctl{abort_flag, p.status};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&kv_map);
+            prefetch_tensormap(&q_map);
+            run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) run_mma<NG>(p, meta, bginfo, smem, tmem, ctl);
+    } else {
+        run_softmax<NG>(p, meta, bginfo, smem, tmem, ctl);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+// LSE-weighted merge of split partials; one CTA per (request, head group).
+__global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombineParams p) {
+    const int bg = blockIdx.x;
+    const int32_t* hdr = p.sched;
+    if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
+        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != p.NG) {
+        if (threadIdx.x == 0 && bg == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        return;
+    }
+    const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
+    const int base = __ldg(info + 0);
+    const int k = __ldg(info + 1);
+    if (k == 1) return;
+    if (k > 1 && (base < 0 || base + k > p.slots_cap)) {
+        if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        return;
+    }
+    const int b = bg / p.Hg;
+    const int g = bg - b * p.Hg;
+    const int d0 = threadIdx.x * 4;
+    for (int n = 0; n < p.NG; ++n) {
+        const int gc = g * p.NG + n;
+        if (gc >= p.N) break;
+        const int s = gc / p.heads;
+        const int head = gc - s * p.heads;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lstar = -INFINITY;
+        if (k > 1) {
+            float mx = -INFINITY;
+            for (int i = 0; i < k; ++i) mx = fmaxf(mx, __ldg(p.lpart + (size_t)(base + i) * p.NG + n));
+            if (mx != -INFINITY) {
+                float sum = 0.f;
+                for (int i = 0; i < k; ++i) sum += expf(__ldg(p.lpart + (size_t)(base + i) * p.NG + n) - mx);
+                lstar = mx + logf(sum);
+                for (int i = 0; i < k; ++i) {
+                    const float w = expf(__ldg(p.lpart + (size_t)(base + i) * p.NG + n) - lstar);
+                    const float4 v = __ldg(reinterpret_cast<const float4*>(
+                        p.opart + ((size_t)(base + i) * p.NG + n) * kDv + d0));
+                    acc.x += w * v.x;
+                    acc.y += w * v.y;
+                    acc.z += w * v.z;
+                    acc.w += w * v.w;
+                }
+            }
+        }
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 packed;
+        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(p.out + (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0) = packed;
+        if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
+    }
+}
+
+// Block-wide inclusive scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int r = v + (warp > 0 ? warp_tot[warp - 1] : 0);
+    __syncthreads();
+    return r;
+}
+
+// Builds the persistent-CTA plan on the device (one block of 1024 threads).
+__global__ void __launch_bounds__(1024)
+    mla_decode_schedule_kernel(const int32_t* __restrict__ seqlens, int32_t* __restrict__ sched, int B,
+                               int Hg, int NG, int G, int max_blocks) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    __shared__ int bad_len;
+    const int BG = B * Hg;
+    int32_t* prefix = sched + prefix_offset_words(G, BG);
+    int32_t* bginfo = sched + bg_offset_words(G);
+    int32_t* meta = sched + kHdrWords;
+    if (threadIdx.x == 0) {
+        carry = 0;
+        bad_len = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < BG; base += 1024) {
+        const int bg = base + threadIdx.x;
+        int v = 0;
+        if (bg < BG) {
+            const int L = seqlens[bg / Hg];
+            if (!seqlen_in_range(L, max_blocks)) bad_len = 1;
+            v = (int)units_of(pages_of(clamp_seqlen(L, max_blocks)));
+        }
+        const int incl = block_inclusive_scan(v, warp_tot);
+        if (bg < BG) prefix[bg] = carry + incl - v;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry += incl;
+        __syncthreads();
+    }
+    const int64_t W = carry;
+    if (threadIdx.x == 0) prefix[BG] = (int)W;
+    __syncthreads();
+    const int64_t T = units_per_cta(W, G);
+    for (int k = threadIdx.x; k < G; k += 1024)
+        cta_meta(prefix, BG, W, T, k, seqlens, Hg, max_blocks, meta + (size_t)k * kMetaWords);
+    __syncthreads();
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < BG; base += 1024) {
+        const int bg = base + threadIdx.x;
+        int ns = 0;
+        if (bg < BG) ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, max_blocks), T);
+        const int v = ns > 1 ? ns : 0;
+        const int incl = block_inclusive_scan(v, warp_tot);
+        if (bg < BG) {
+            bginfo[kBgWords * bg] = carry + incl - v;
+            bginfo[kBgWords * bg + 1] = ns;
+        }
+        __syncthreads();
+        if (threadIdx.x == 1023) carry += incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        sched[kHdrMagic] = kSchedMagic;
+        sched[kHdrG] = G;
+        sched[kHdrBG] = BG;
+        sched[kHdrHg] = Hg;
+        sched[kHdrNG] = NG;
+        sched[kHdrSlots] = carry;
+        sched[kHdrT] = (int)T;
+        sched[kHdrStatus] = bad_len ? MLA_STATUS_BAD_SEQLEN : 0;
+        sched[kHdrW] = (int)W;
+        sched[kHdrBatch] = B;
+        sched[kHdrMaxBlocks] = max_blocks;
+        for (int i = kHdrMaxBlocks + 1; i < kHdrWords; ++i) sched[i] = 0;
+    }
+}
+
+}  // namespace mla

@@ -1,0 +1,318 @@
+// C ABI of the sm_100a MLA decode library: argument checks, TMA tensor maps,
+// launches.  Declarations and their contract: include/mla_decode.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "decode_kernels.cuh"
+#include "mla_decode.h"
+#include "schedule.cuh"
+
+namespace {
+
+using namespace mla;
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxDevices = 64;
+
+int validate_dims(const mla_decode_dims* d) {
+    if (d == nullptr) return MLA_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->s_q < 1 || d->num_heads < 1 || d->num_blocks < 1 ||
+        d->max_blocks_per_seq < 1 || d->num_sms < 0 || d->reserved != 0 ||
+        (d->flags & ~MLA_FLAG_NO_COMBINE) != 0 || (d->causal != 0 && d->causal != 1))
+        return MLA_ERR_INVALID_ARG;
+    if (d->page_size != kPage || d->d_qk != kDqk || d->d_v != kDv) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)d->num_heads * d->s_q > 256) return MLA_ERR_UNSUPPORTED;
+    const Grouping gr = make_grouping(d->num_heads, d->s_q);
+    const int64_t BG = (int64_t)d->batch * gr.Hg;
+    // Work units and row counts must fit the int32 arithmetic of the kernels.
+    if (BG * ((int64_t)d->max_blocks_per_seq + kItemOverhead) >= (int64_t)INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * gr.N >= (int64_t)INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * d->max_blocks_per_seq >= (int64_t)INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+int resolve_ctas(const mla_decode_dims* d, int* G) {
+    if (d->num_sms > 0) {
+        *G = d->num_sms;
+        return MLA_OK;
+    }
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    *G = n;
+    return MLA_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Plan {
+    Grouping gr;
+    int G;
+    int BG;
+    int64_t slots;
+};
+
+int make_plan(const mla_decode_dims* d, Plan* pl) {
+    int rc = validate_dims(d);
+    if (rc != MLA_OK) return rc;
+    rc = resolve_ctas(d, &pl->G);
+    if (rc != MLA_OK) return rc;
+    pl->gr = make_grouping(d->num_heads, d->s_q);
+    pl->BG = d->batch * pl->gr.Hg;
+    pl->slots = max_slots(pl->G);
+    return MLA_OK;
+}
+
+size_t workspace_bytes_of(const Plan& pl) {
+    const size_t per_slot = (size_t)pl.gr.NG * (kDv + 1) * sizeof(float);
+    return (size_t)pl.slots * per_slot;
+}
+
+// ---- TMA tensor maps ----
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Pool [num_blocks][64][576] bf16 viewed as 3-D (col, token, page); box = 64 cols x 64 tokens.
+int make_kv_map(CUtensorMap* m, const void* kv, int num_blocks) {
+    auto enc = get_encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)kDqk, (cuuint64_t)kPage, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)kDqk * 2, (cuuint64_t)kDqk * 2 * kPage};
+    cuuint32_t box[3] = {64, (cuuint32_t)kPage, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Q [B*s_q*h][576] bf16 as 2-D; box = 64 cols x NG rows (rows past the end read as zero).
+int make_q_map(CUtensorMap* m, const void* q, int rows, int NG) {
+    auto enc = get_encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)kDqk, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kDqk * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)NG};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <int NG>
+int ensure_smem_attr() {
+    static bool done[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(mla_decode_fwd_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FwdSmem<NG>::kAlloc) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        done[dev] = true;
+    }
+    return MLA_OK;
+}
+
+template <int NG>
+int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const CUtensorMap& qm,
+               cudaStream_t stream) {
+    int rc = ensure_smem_attr<NG>();
+    if (rc != MLA_OK) return rc;
+    mla_decode_fwd_kernel<NG><<<pl.G, kFwdThreads, FwdSmem<NG>::kAlloc, stream>>>(kvm, qm, p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedule, const void* workspace,
+                   void* out, float* lse, cudaStream_t stream) {
+    CombineParams c;
+    c.sched = static_cast<const int32_t*>(schedule);
+    c.opart = static_cast<const float*>(workspace);
+    c.lpart = c.opart + (size_t)pl.slots * pl.gr.NG * kDv;
+    c.out = static_cast<__nv_bfloat16*>(out);
+    c.lse = lse;
+    c.status = const_cast<int32_t*>(c.sched) + kHdrStatus;
+    c.s_q = d->s_q;
+    c.heads = d->num_heads;
+    c.N = pl.gr.N;
+    c.NG = pl.gr.NG;
+    c.Hg = pl.gr.Hg;
+    c.G = pl.G;
+    c.BG = pl.BG;
+    c.slots_cap = (int)pl.slots;
+    mla_decode_combine_kernel<<<pl.BG, 128, 0, stream>>>(c);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_version(void) { return kAbiVersion; }
+
+const char* mla_decode_strerror(int code) {
+    switch (code) {
+        case MLA_OK: return "ok";
+        case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or bad dims)";
+        case MLA_ERR_UNSUPPORTED: return "unsupported shape (page_size must be 64, d_qk 576, d_v 512, heads*s_q <= 256)";
+        case MLA_ERR_CUDA: return "CUDA runtime or launch error";
+        case MLA_ERR_BAD_SCHEDULE: return "schedule buffer does not match these dims";
+        default: return "unknown error code";
+    }
+}
+
+size_t mla_decode_schedule_bytes(const mla_decode_dims* dims) {
+    Plan pl;
+    if (make_plan(dims, &pl) != MLA_OK) return 0;
+    return (size_t)schedule_words(pl.G, pl.BG) * sizeof(int32_t);
+}
+
+size_t mla_decode_workspace_bytes(const mla_decode_dims* dims) {
+    Plan pl;
+    if (make_plan(dims, &pl) != MLA_OK) return 0;
+    return workspace_bytes_of(pl);
+}
+
+int mla_decode_get_schedule(const mla_decode_dims* dims, const int32_t* cache_seqlens, void* schedule,
+                            void* stream) {
+    Plan pl;
+    int rc = make_plan(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
+    mla_decode_schedule_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.gr.Hg, pl.gr.NG, pl.G,
+        dims->max_blocks_per_seq);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seqlens, void* schedule_host) {
+    int rc = validate_dims(dims);
+    if (rc != MLA_OK) return rc;
+    if (dims->num_sms <= 0 || seqlens == nullptr || schedule_host == nullptr) return MLA_ERR_INVALID_ARG;
+    const Grouping gr = make_grouping(dims->num_heads, dims->s_q);
+    const int G = dims->num_sms, BG = dims->batch * gr.Hg, mb = dims->max_blocks_per_seq;
+    int32_t* s = static_cast<int32_t*>(schedule_host);
+    int32_t* prefix = s + prefix_offset_words(G, BG);
+    int32_t* bginfo = s + bg_offset_words(G);
+    int bad_len = 0;
+    int64_t W = 0;
+    for (int bg = 0; bg < BG; ++bg) {
+        const int L = seqlens[bg / gr.Hg];
+        if (!seqlen_in_range(L, mb)) bad_len = 1;
+        prefix[bg] = (int32_t)W;
+        W += units_of(pages_of(clamp_seqlen(L, mb)));
+    }
+    prefix[BG] = (int32_t)W;
+    const int64_t T = units_per_cta(W, G);
+    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, seqlens, gr.Hg, mb, s + kHdrWords + (size_t)k * kMetaWords);
+    int64_t slots = 0;
+    for (int bg = 0; bg < BG; ++bg) {
+        const int ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, gr.Hg, mb), T);
+        bginfo[kBgWords * bg] = (int32_t)slots;
+        bginfo[kBgWords * bg + 1] = ns;
+        if (ns > 1) slots += ns;
+    }
+    std::memset(s, 0, kHdrWords * sizeof(int32_t));
+    s[kHdrMagic] = kSchedMagic;
+    s[kHdrG] = G;
+    s[kHdrBG] = BG;
+    s[kHdrHg] = gr.Hg;
+    s[kHdrNG] = gr.NG;
+    s[kHdrSlots] = (int32_t)slots;
+    s[kHdrT] = (int32_t)T;
+    s[kHdrStatus] = bad_len ? MLA_STATUS_BAD_SEQLEN : 0;
+    s[kHdrW] = (int32_t)W;
+    s[kHdrBatch] = dims->batch;
+    s[kHdrMaxBlocks] = mb;
+    return MLA_OK;
+}
+
+int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* workspace, const void* q,
+                   const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
+                   float softmax_scale, void* out, float* lse, void* stream) {
+    Plan pl;
+    int rc = make_plan(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(q) || !aligned16(kv_cache) ||
+        !aligned16(block_table) || !aligned16(cache_seqlens) || !aligned16(out) || !aligned16(lse))
+        return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    CUtensorMap kvm, qm;
+    rc = make_kv_map(&kvm, kv_cache, dims->num_blocks);
+    if (rc != MLA_OK) return rc;
+    rc = make_q_map(&qm, q, dims->batch * pl.gr.N, pl.gr.NG);
+    if (rc != MLA_OK) return rc;
+    FwdParams p;
+    p.sched = static_cast<const int32_t*>(schedule);
+    p.block_table = block_table;
+    p.seqlens = cache_seqlens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.opart = static_cast<float*>(workspace);
+    p.lpart = p.opart + (size_t)pl.slots * pl.gr.NG * kDv;
+    p.status = const_cast<int32_t*>(p.sched) + kHdrStatus;
+    p.s_q = dims->s_q;
+    p.heads = dims->num_heads;
+    p.N = pl.gr.N;
+    p.num_blocks = dims->num_blocks;
+    p.max_blocks = dims->max_blocks_per_seq;
+    p.causal = dims->causal;
+    p.G = pl.G;
+    p.BG = pl.BG;
+    p.Hg = pl.gr.Hg;
+    p.slots_cap = (int)pl.slots;
+    p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = pl.gr.NG == 16 ? launch_fwd<16>(pl, p, kvm, qm, st) : launch_fwd<32>(pl, p, kvm, qm, st);
+    if (rc != MLA_OK) return rc;
+    if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
+    return launch_combine(dims, pl, schedule, workspace, out, lse, st);
+}
+
+int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const void* workspace, void* out,
+                       float* lse, void* stream) {
+    Plan pl;
+    int rc = make_plan(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
+        return MLA_ERR_INVALID_ARG;
+    return launch_combine(dims, pl, schedule, workspace, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_get_status(const void* schedule, int32_t* host_status) {
+    if (!aligned16(schedule) || host_status == nullptr) return MLA_ERR_INVALID_ARG;
+    const int32_t* src = static_cast<const int32_t*>(schedule) + kHdrStatus;
+    if (cudaMemcpy(host_status, src, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+}  // extern "C"

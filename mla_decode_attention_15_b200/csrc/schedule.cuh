@@ -1,0 +1,177 @@
+// Split-KV work partitioning for the persistent decode kernel.
+//
+// Work units: request b, head group g ("bg" = b * Hg + g) owns
+//   units(bg) = P_b + kItemOverhead   (P_b = ceil(L_b / 64) pages; 0 if P_b == 0)
+// The overhead stands for the per-item cost that does not scale with pages:
+// loading Q, filling the pipeline, the epilogue.  Units are laid out in bg
+// order and cut into G equal contiguous ranges of T units; CTA k owns
+// [k*T, (k+1)*T).  A unit position u inside bg maps to page
+// clamp(u - start(bg) - overhead, 0, P_b), so a CTA's range is a list of
+// (bg, page range) items; only its first and last item can be partial, and a
+// bg covered by more than one CTA is "split": each piece writes an fp32
+// partial that the combine kernel merges by LSE weight.
+//
+// The pages describe no scheduler; this greedy contiguous partition is the
+// plainest one that balances ragged lengths across the SMs.
+#pragma once
+
+#include <cstdint>
+
+#include "mla_decode.h"
+
+namespace mla {
+
+constexpr int kPage = 64;
+constexpr int kDqk = 576;
+constexpr int kDv = 512;
+constexpr int kItemOverhead = 1;   // units charged per (request, head group)
+constexpr int kMinPagesPerCta = 2; // smallest range worth its own CTA
+
+// ---- schedule buffer layout (int32 words) ----
+constexpr int kSchedMagic = 0x4D4C4144;  // 'MLAD'
+constexpr int kHdrWords = 16;
+enum HdrField {
+    kHdrMagic = 0,
+    kHdrG = 1,
+    kHdrBG = 2,
+    kHdrHg = 3,
+    kHdrNG = 4,
+    kHdrSlots = 5,
+    kHdrT = 6,
+    kHdrStatus = 7,
+    kHdrW = 8,
+    kHdrBatch = 9,
+    kHdrMaxBlocks = 10,
+};
+constexpr int kMetaWords = 8;  // per CTA: begin_bg, begin_page, end_bg, end_page, first_split
+enum MetaField { kMetaBeginBg = 0, kMetaBeginPage = 1, kMetaEndBg = 2, kMetaEndPage = 3, kMetaFirstSplit = 4 };
+constexpr int kBgWords = 2;  // per bg: slot_base, num_splits
+
+__host__ __device__ inline int64_t meta_offset_words() { return kHdrWords; }
+__host__ __device__ inline int64_t bg_offset_words(int G) { return kHdrWords + (int64_t)kMetaWords * G; }
+__host__ __device__ inline int64_t prefix_offset_words(int G, int BG) {
+    return bg_offset_words(G) + (int64_t)kBgWords * BG;
+}
+__host__ __device__ inline int64_t schedule_words(int G, int BG) {
+    return prefix_offset_words(G, BG) + BG + 1;
+}
+
+// Head grouping: N = heads * s_q query columns per request.  Up to 32 columns
+// go in one group (rounded up to 16 / 32 for the MMA N); more are cut into
+// groups of 32.
+struct Grouping {
+    int N;   // heads * s_q
+    int NG;  // columns per group (MMA N): 16 or 32
+    int Hg;  // groups per request
+};
+__host__ __device__ inline Grouping make_grouping(int heads, int s_q) {
+    Grouping gr;
+    gr.N = heads * s_q;
+    if (gr.N <= 16) {
+        gr.NG = 16;
+        gr.Hg = 1;
+    } else if (gr.N <= 32) {
+        gr.NG = 32;
+        gr.Hg = 1;
+    } else {
+        gr.NG = 32;
+        gr.Hg = (gr.N + 31) / 32;
+    }
+    return gr;
+}
+
+// Cached length clamped to what the block table can address.
+__host__ __device__ inline int clamp_seqlen(int L, int max_blocks) {
+    int64_t cap = (int64_t)max_blocks * kPage;
+    if (L < 0) return 0;
+    if ((int64_t)L > cap) return (int)cap;
+    return L;
+}
+__host__ __device__ inline bool seqlen_in_range(int L, int max_blocks) {
+    return L >= 0 && (int64_t)L <= (int64_t)max_blocks * kPage;
+}
+__host__ __device__ inline int pages_of(int L) { return (L + kPage - 1) / kPage; }
+__host__ __device__ inline int64_t units_of(int P) { return P > 0 ? (int64_t)P + kItemOverhead : 0; }
+
+__host__ __device__ inline int64_t units_per_cta(int64_t W, int G) {
+    int64_t T = (W + G - 1) / (G > 0 ? G : 1);
+    int64_t lo = kMinPagesPerCta + kItemOverhead;
+    return T < lo ? lo : T;
+}
+
+// Largest bg in [0, BG) with prefix[bg] <= u (prefix non-decreasing, prefix[0] == 0).
+__host__ __device__ inline int find_bg(const int32_t* prefix, int BG, int64_t u) {
+    int lo = 0, hi = BG - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Pages of request-group bg under the clamp every kernel applies.
+__host__ __device__ inline int pages_of_bg(const int32_t* seqlens, int bg, int Hg, int max_blocks) {
+    return pages_of(clamp_seqlen(seqlens[bg / Hg], max_blocks));
+}
+
+// (bg, page) position of unit u; u >= W maps to (BG, 0).
+__host__ __device__ inline void locate_unit(const int32_t* prefix, int BG, int64_t W, int64_t u,
+                                            const int32_t* seqlens, int Hg, int max_blocks,
+                                            int* bg_out, int* page_out) {
+    if (u >= W) {
+        *bg_out = BG;
+        *page_out = 0;
+        return;
+    }
+    int bg = find_bg(prefix, BG, u);
+    int P = pages_of_bg(seqlens, bg, Hg, max_blocks);
+    int64_t p = u - (int64_t)prefix[bg] - kItemOverhead;
+    if (p < 0) p = 0;
+    if (p > P) p = P;
+    *bg_out = bg;
+    *page_out = (int)p;
+}
+
+// First / last CTA that owns a page of bg (P > 0).
+__host__ __device__ inline int first_cta_of(const int32_t* prefix, int bg, int64_t T) {
+    return (int)(((int64_t)prefix[bg] + kItemOverhead) / T);
+}
+__host__ __device__ inline int last_cta_of(const int32_t* prefix, int bg, int P, int64_t T) {
+    return (int)(((int64_t)prefix[bg] + kItemOverhead + P - 1) / T);
+}
+
+__host__ __device__ inline int num_splits_of(const int32_t* prefix, int bg, int P, int64_t T) {
+    return P > 0 ? last_cta_of(prefix, bg, P, T) - first_cta_of(prefix, bg, T) + 1 : 0;
+}
+
+// Work range of CTA k: units [k*T, min((k+1)*T, W)).
+__host__ __device__ inline void cta_meta(const int32_t* prefix, int BG, int64_t W, int64_t T, int k,
+                                         const int32_t* seqlens, int Hg, int max_blocks,
+                                         int32_t* meta) {
+    int64_t u0 = (int64_t)k * T;
+    int64_t u1 = u0 + T;
+    if (u0 > W) u0 = W;
+    if (u1 > W) u1 = W;
+    int bb, bp, eb, ep;
+    locate_unit(prefix, BG, W, u0, seqlens, Hg, max_blocks, &bb, &bp);
+    locate_unit(prefix, BG, W, u1, seqlens, Hg, max_blocks, &eb, &ep);
+    int first_split = 0;
+    if (bb < BG) {
+        int P = pages_of_bg(seqlens, bb, Hg, max_blocks);
+        if (P > 0) {
+            first_split = k - first_cta_of(prefix, bb, T);
+            if (first_split < 0) first_split = 0;
+        }
+    }
+    meta[kMetaBeginBg] = bb;
+    meta[kMetaBeginPage] = bp;
+    meta[kMetaEndBg] = eb;
+    meta[kMetaEndPage] = ep;
+    meta[kMetaFirstSplit] = first_split;
+    meta[5] = meta[6] = meta[7] = 0;
+}
+
+// Upper bound of partial slots: every CTA has at most two partial items.
+__host__ __device__ inline int64_t max_slots(int G) { return 2 * (int64_t)G; }
+
+}  // namespace mla

@@ -1,0 +1,184 @@
+"""GPU parity: the sm_100a decode path (called through the C ABI) against the
+fp64 oracle on identical seeded inputs.
+
+Tolerances (see helpers.py): max|err| <= 1e-2 max|O_ref|, RMSE <= 5e-4 (plus
+the bf16 rounding floor of the exact result where that floor exceeds 2.5e-4,
+i.e. on peaked rows), |dLSE| <= 1e-5 max(1, |LSE|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import helpers
+import oracle
+from mla_decode_attention_15_b200 import _build, binding as bd, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    major, _ = torch.cuda.get_device_capability(0)
+    assert major == 10, "the library is built for sm_100a (B200)"
+    _build.build()
+    bd.lib()
+    oracle.build()
+    return torch.device("cuda:0")
+
+
+def to_dev(d, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def run_gpu(d, dev, num_sms=0, flags=0, expect_status=0):
+    g = to_dev(d, dev)
+    B, s_q, h, _ = g["q"].shape
+    dec = bd.MlaDecoder(B, s_q, h, g["kv_cache"].shape[0], g["block_table"].shape[1], g["causal"],
+                        num_sms, dev)
+    if flags:
+        dec.dims.flags = flags
+    dec.plan(g["cache_seqlens"])
+    out, lse = dec(g["q"], g["kv_cache"], g["block_table"], g["cache_seqlens"], g["softmax_scale"])
+    if flags & bd.MLA_FLAG_NO_COMBINE:
+        bd.mla_decode_combine(dec.dims, dec.schedule, dec.workspace, dec.out, dec.lse)
+    torch.cuda.synchronize()
+    assert dec.status() == expect_status
+    return out.clone(), lse.clone(), dec
+
+
+def ref(d, rows=None):
+    return oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                 d["softmax_scale"], causal=d["causal"], rows=rows)
+
+
+def check(d, dev, rows=None, **kw):
+    out, lse, _ = run_gpu(d, dev, **kw)
+    ro, rl = ref(d, rows)
+    return helpers.compare(out, lse, ro, rl, rows=rows)
+
+
+# ------------------------------------------------------------------ schedule
+@pytest.mark.parametrize("lens,heads,s_q", [
+    ([1024], 16, 1), ([4096] * 16, 16, 1), ([0, 5, 64, 65, 9000, 1, 130], 16, 2),
+    ([20000, 8192, 32768, 100], 128, 2), ([65536] * 16, 16, 1)])
+def test_device_schedule_matches_host(dev, lens, heads, s_q):
+    sl = torch.tensor(lens, dtype=torch.int32)
+    mb = max(1, (max(lens) + 63) // 64)
+    dims = bd.make_dims(len(lens), s_q, heads, 10 ** 6, mb, True, 148)
+    n = bd.mla_decode_schedule_bytes(dims)
+    host = torch.zeros(n, dtype=torch.uint8)
+    bd.mla_decode_get_schedule_host(dims, sl, host)
+    devbuf = torch.full((n,), 0xAB, dtype=torch.uint8, device=dev)
+    bd.mla_decode_get_schedule(dims, sl.to(dev), devbuf)
+    torch.cuda.synchronize()
+    assert torch.equal(devbuf.cpu(), host)
+
+
+# ------------------------------------------------------------------ workloads
+@pytest.mark.parametrize("name", ["b1_l1024_h16", "b16_l4096_h16", "b16_sq2_ragged1k16k_h16_peaked"])
+def test_workload_all_outputs(dev, name):
+    d = workloads.make_inputs(name)
+    m = check(d, dev)
+    print(name, m)
+
+
+def test_headline_sampled_outputs(dev):
+    """batch 16 x 64K: the launch bench.py times, checked on sampled rows."""
+    d = workloads.make_inputs("b16_l65536_h16")
+    out, lse, _ = run_gpu(d, dev)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    rng = np.random.default_rng(0)
+    rows = sorted(set(int(b) * 16 + int(h) for b, h in zip(rng.integers(0, 16, 24), rng.integers(0, 16, 24))))
+    ro, rl = ref(d, rows)
+    m = helpers.compare(out, lse, ro, rl, rows=rows)
+    print(m)
+
+
+def test_wide_heads_sampled_outputs(dev):
+    """batch 32, s_q 2 causal, 128 heads (8 head groups of 32 columns)."""
+    d = workloads.make_inputs("b32_sq2_ragged8k32k_h128")
+    out, lse, _ = run_gpu(d, dev)
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(1)
+    B, s_q, h = 32, 2, 128
+    rows = sorted(set(int(x) for x in rng.integers(0, B * s_q * h, 40)))
+    ro, rl = ref(d, rows)
+    m = helpers.compare(out, lse, ro, rl, rows=rows)
+    print(m)
+
+
+# ------------------------------------------------------------------ edge cases
+@pytest.mark.parametrize("s_q,causal", [(1, False), (2, True), (2, False)])
+@pytest.mark.parametrize("num_sms", [1, 3, 148])
+def test_ragged_tails_and_splits(dev, s_q, causal, num_sms):
+    lens = [1, 2, 63, 64, 65, 127, 128, 130, 1000, 4099]
+    d = workloads.build(len(lens), s_q, 16, ("list", lens), seed=21 + num_sms, causal=causal)
+    check(d, dev, num_sms=num_sms)
+
+
+@pytest.mark.parametrize("heads,s_q", [(1, 1), (3, 2), (8, 2), (24, 2), (40, 1), (128, 2), (128, 1)])
+def test_head_counts(dev, heads, s_q):
+    lens = [300, 77, 1025]
+    d = workloads.build(len(lens), s_q, heads, ("list", lens), seed=31 + heads, causal=(s_q > 1))
+    check(d, dev)
+
+
+def test_empty_and_short_causal(dev):
+    lens = [0, 1, 2, 0, 70]
+    d = workloads.build(len(lens), 2, 16, ("list", lens), seed=41, causal=True)
+    out, lse, _ = run_gpu(d, dev)
+    ro, rl = ref(d)
+    helpers.compare(out, lse, ro, rl)
+    assert (out[0] == 0).all() and torch.isneginf(lse[0]).all()
+    assert torch.isneginf(lse[1, :, 0]).all()   # L = 1: token 0 sees nothing
+
+
+def test_rows_past_length_do_not_matter(dev):
+    lens = [65, 1000, 129]
+    d = workloads.build(len(lens), 2, 16, ("list", lens), seed=51, causal=True, tail_fill=1e4)
+    check(d, dev, num_sms=5)
+
+
+def test_identity_and_permuted_tables_agree(dev):
+    a = workloads.build(2, 1, 16, ("list", [700, 1300]), seed=61, table="identity")
+    b = dict(a)
+    perm = torch.randperm(a["kv_cache"].shape[0], generator=torch.Generator().manual_seed(1))
+    inv = torch.argsort(perm)
+    b["kv_cache"] = a["kv_cache"][perm].contiguous()
+    bt = a["block_table"].clone()
+    bt[bt >= 0] = inv[bt[bt >= 0].long()].to(torch.int32)
+    b["block_table"] = bt
+    oa, la, _ = run_gpu(a, dev)
+    ob, lb, _ = run_gpu(b, dev)
+    assert torch.equal(oa, ob) and torch.equal(la, lb)
+
+
+def test_repeat_runs_are_bitwise_identical(dev):
+    d = workloads.make_inputs("b16_sq2_ragged1k16k_h16_peaked")
+    o1, l1, _ = run_gpu(d, dev)
+    o2, l2, _ = run_gpu(d, dev)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_explicit_combine_matches_fused_launch(dev):
+    d = workloads.build(3, 1, 16, ("list", [5000, 64, 2222]), seed=71)
+    o1, l1, _ = run_gpu(d, dev, num_sms=16)
+    o2, l2, _ = run_gpu(d, dev, num_sms=16, flags=bd.MLA_FLAG_NO_COMBINE)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_single_cta_walks_many_items(dev):
+    lens = [130, 1, 64, 900, 65, 3, 2048, 640]
+    d = workloads.build(len(lens), 2, 16, ("list", lens), seed=81, causal=True)
+    check(d, dev, num_sms=1)
+
+
+def test_bad_block_table_is_reported_not_faulted(dev):
+    d = workloads.build(2, 1, 16, ("list", [300, 200]), seed=91)
+    d["block_table"] = d["block_table"].clone()
+    d["block_table"][1, 2] = 10 ** 6
+    out, lse, dec = run_gpu(d, dev, expect_status=bd.MLA_STATUS_BAD_BLOCK_TABLE)
+    # the device stays usable and a clean run reports no fault
+    good = workloads.build(1, 1, 16, ("list", [100]), seed=92)
+    check(good, dev)

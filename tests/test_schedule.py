@@ -1,0 +1,121 @@
+"""Integer invariants of the split-KV plan, computed on the host by
+mla_decode_get_schedule_host (the same plan the device kernel builds; a GPU
+test checks the two are bit-identical)."""
+import numpy as np
+import pytest
+import torch
+
+import helpers
+from mla_decode_attention_15_b200 import _build, binding as bd, workloads
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    _build.build()
+    bd.lib()
+
+
+def host_plan(seqlens, s_q, heads, G, max_blocks=None):
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int32).contiguous()
+    B = seqlens.numel()
+    if max_blocks is None:
+        max_blocks = max(1, (int(seqlens.clamp(min=0).max()) + 63) // 64)
+    d = bd.make_dims(B, s_q, heads, 10 ** 6, max_blocks, False, G)
+    n = bd.mla_decode_schedule_bytes(d)
+    buf = torch.zeros(n, dtype=torch.uint8)
+    bd.mla_decode_get_schedule_host(d, seqlens, buf)
+    Hg = 1 if heads * s_q <= 32 else (heads * s_q + 31) // 32
+    BG = B * Hg
+    hdr, meta, bginfo, prefix = helpers.read_plan(buf.numpy(), G, BG)
+    return dict(hdr=hdr, meta=meta, bginfo=bginfo, prefix=prefix, Hg=Hg, BG=BG, G=G,
+                seqlens=seqlens.numpy(), max_blocks=max_blocks)
+
+
+def check_invariants(pl):
+    seq, Hg, BG, G, mb = pl["seqlens"], pl["Hg"], pl["BG"], pl["G"], pl["max_blocks"]
+    hdr, meta, bginfo = pl["hdr"], pl["meta"], pl["bginfo"]
+    assert hdr[0] == 0x4D4C4144 and hdr[1] == G and hdr[2] == BG and hdr[3] == Hg
+    T = int(hdr[6])
+    items = helpers.walk_plan(meta, bginfo, seq, Hg, mb)
+    pages = [(min(max(int(seq[bg // Hg]), 0), mb * 64) + 63) // 64 for bg in range(BG)]
+    covered = [np.zeros(P, dtype=np.int64) for P in pages]
+    pieces = [[] for _ in range(BG)]
+    for k, its in enumerate(items):
+        load = 0
+        for (bg, p0, p1, unsplit, slot) in its:
+            covered[bg][p0:p1] += 1
+            pieces[bg].append((k, p0, p1, unsplit, slot))
+            load += (p1 - p0)
+        # a CTA never carries more than its share of units (pages + 1 per item)
+        assert load + len(its) * helpers.OVERHEAD <= T + helpers.OVERHEAD, (k, its, T)
+        # only the first and the last item of a CTA can be partial
+        for (bg, p0, p1, unsplit, slot) in its[1:-1]:
+            assert unsplit
+    for bg in range(BG):
+        assert (covered[bg] == 1).all(), bg  # every page exactly once
+        ns = int(bginfo[bg, 1])
+        assert ns == len(pieces[bg]), (bg, ns, pieces[bg])
+        if ns == 1:
+            assert pieces[bg][0][3]  # unsplit, written directly
+        if ns > 1:
+            slots = sorted(pc[4] for pc in pieces[bg])
+            base = int(bginfo[bg, 0])
+            assert slots == list(range(base, base + ns))
+            assert not any(pc[3] for pc in pieces[bg])
+    total_slots = sum(int(bginfo[bg, 1]) for bg in range(BG) if bginfo[bg, 1] > 1)
+    assert total_slots == int(hdr[5]) <= 2 * G
+    return items
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_plan_of_each_workload(name):
+    w = workloads.WORKLOADS[name]
+    g = torch.Generator().manual_seed(w.seed)
+    if w.lens[0] == "fixed":
+        lens = [w.lens[1]] * w.batch
+    else:
+        lens = torch.randint(w.lens[1], w.lens[2] + 1, (w.batch,), generator=g).tolist()
+    pl = host_plan(lens, w.s_q, w.heads, 148)
+    items = check_invariants(pl)
+    busy = sum(1 for its in items if its)
+    W = int(pl["hdr"][8])
+    assert busy == min(148, -(-W // int(pl["hdr"][6])))
+
+
+@pytest.mark.parametrize("G", [1, 2, 7, 148, 300])
+@pytest.mark.parametrize("heads,s_q", [(16, 1), (16, 2), (1, 1), (3, 2), (24, 2), (128, 2)])
+def test_plan_random_ragged(G, heads, s_q):
+    rng = np.random.default_rng(G * 1000 + heads * 10 + s_q)
+    lens = rng.integers(0, 3000, size=int(rng.integers(1, 40))).tolist()
+    lens[0] = 0
+    check_invariants(host_plan(lens, s_q, heads, G))
+
+
+def test_plan_long_single_request_spreads_over_all_ctas():
+    pl = host_plan([65536], 1, 16, 148)
+    items = check_invariants(pl)
+    busy = [its for its in items if its]
+    assert all(len(its) == 1 for its in busy)
+    T = int(pl["hdr"][6])
+    assert T == -(-(1024 + 1) // 148)
+    assert len(busy) == -(-(1024 + 1) // T) >= 140
+    assert int(pl["bginfo"][0, 1]) == len(busy)
+
+
+def test_plan_short_batch_uses_few_ctas():
+    pl = host_plan([1024], 1, 16, 148)  # 16 pages
+    items = check_invariants(pl)
+    busy = [its for its in items if its]
+    assert 2 <= len(busy) <= 8
+    assert all(p1 - p0 >= 1 for its in busy for (_, p0, p1, _, _) in its)
+
+
+def test_plan_clamps_and_flags_bad_lengths():
+    pl = host_plan([100, -5, 10 ** 6], 1, 16, 8, max_blocks=4)
+    assert pl["hdr"][7] & bd.MLA_STATUS_BAD_SEQLEN
+    items = check_invariants(pl)
+    assert int(pl["bginfo"][1, 1]) == 0          # negative length: empty request
+    total = sum(p1 - p0 for its in items for (bg, p0, p1, _, _) in its if bg == 2)
+    assert total == 4                            # clamped to the table's 4 pages
+    ok = host_plan([100, 5], 1, 16, 8, max_blocks=4)
+    assert ok["hdr"][7] == 0
