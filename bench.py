@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0,
+                    help="decode only the first BATCH requests of the workload (small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -456,6 +458,10 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
 def main():
     args = parse_args()
     w = workloads.WORKLOADS[args.workload]
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.batch,
+                                description=w.description + "; first %d requests only" % args.batch)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -14,12 +14,16 @@
 //   warp 0        TMA producer: Q of the work item, then every 64-token page
 //                 gathered through the block table (9 boxes of 64x64 bf16,
 //                 128-byte swizzle) into a 2-stage ring of 72 KB stages.
-//   warp 1        one thread issues tcgen05.mma:
-//                   GEMM1  S^T[64 x N]  = K[64 x 576] . Q^T        (M=64, K-major A and B)
-//                   GEMM2  O^T[512 x N] += V^T[512 x 64] . P^T     (4 x M=128, MN-major A and B)
-//                 accumulators live in TMEM; V^T is the same shared-memory page
-//                 read through a second (MN-major) descriptor.
-//   warps 2..5    softmax over the KV axis (one TMEM lane = one token), lazy
+//   warps 1, 2    one thread each issues GEMM1  S^T[64 x N] = K[64 x 576] . Q^T
+//                 (M = 64 tokens, K-major A and B) into TMEM; the two issuers
+//                 take alternate 64-column boxes into separate accumulators,
+//                 which the softmax adds up.
+//   warp 3        one thread issues GEMM2  O^T[512 x N] += V^T[512 x 64] . P^T
+//                 (4 x M = 128 d_v chunks, MN-major A and B); V^T is the same
+//                 shared-memory page read through a second (MN-major) descriptor.
+//                 Separate issuers let GEMM2 of page j start as soon as P^T(j)
+//                 is ready, independently of when page j+1 lands.
+//   warps 4..7    softmax over the KV axis (one TMEM lane = one token), lazy
 //                 rescale of O^T in TMEM, P^T to shared memory as bf16, and the
 //                 epilogue (O = O^T / l transposed back, LSE), either final or
 //                 as an fp32 partial of a split request.
@@ -40,14 +44,80 @@ namespace mla {
 
 constexpr uint32_t kFullMask = 0xffffffffu;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 256;  // 8 warps: TMA, 2 GEMM1 issuers, GEMM2 issuer, 4 softmax
+// A single thread issues at most one tcgen05.mma every ~45 cycles, while the
+// tensor pipe accepts small (M=64, N<=64) MMAs roughly every 28 cycles from two
+// issuers; GEMM1 is therefore issued by two threads (warps 1 and 2), each into
+// its own accumulator, boxes alternating between them.
+constexpr int kG1Issuers = 2;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the running max grows by > 2^8
 constexpr float kLn2 = 0.693147180559945309f;
+// GEMM1 (S^T = K Q^T, K = 576) accumulates into one TMEM accumulator per
+// issuer; the softmax adds them.
+constexpr int kSChains = kG1Issuers;
+
+// L2 prefetch of whole pages ahead of the shared-memory loads
+// (cp.async.bulk.prefetch.L2, one 72 KB page per instruction).  With only two
+// 72 KB stages per SM the refill sees L2 rather than HBM latency (measured on
+// B200: ~1.7 us -> ~1.05 us per page at the bs16 x 64K load).  Short work
+// items gain nothing and lose a little, so only items of at least
+// kPrefetchMinPages pages prefetch.
+#ifndef MLA_PREFETCH_PAGES
+#define MLA_PREFETCH_PAGES 2
+#endif
+constexpr int kPrefetchPages = MLA_PREFETCH_PAGES;
+constexpr int kPrefetchMinPages = 16;
+static_assert(kSChains == kG1Issuers, "one S^T accumulator per GEMM1 issuer");
+
+// Optional timeline tracing (build with -DMLA_TRACE): each role of each CTA
+// stamps %globaltimer at pipeline events into a device buffer that the host
+// copies out with mla_decode_trace_fetch().  Compiled out by default.
+#ifdef MLA_TRACE
+constexpr int kTraceCtas = 160;
+constexpr int kTraceRoles = 4;
+constexpr int kTraceCap = 1024;
+__device__ unsigned long long g_mla_trace[kTraceCtas][kTraceRoles][kTraceCap];
+__device__ unsigned int g_mla_trace_count[kTraceCtas][kTraceRoles];
+enum TraceTag : unsigned {
+    kTrProdIssue = 1,   // producer: stage free, page loads issued
+    kTrMmaKvFull = 2,   // gemm1 issuer: page landed in shared memory
+    kTrMmaPFull = 3,    // gemm2 issuer: P^T ready, GEMM2 about to issue
+    kTrSmSFull = 4,     // softmax: S^T ready in TMEM
+    kTrSmPDone = 5,     // softmax: P^T written (and O rescaled)
+    kTrSmEpi0 = 6,      // softmax: epilogue start (last GEMM2 done)
+    kTrSmEpi1 = 7,      // softmax: epilogue end
+    kTrItem = 8,        // any role: new work item
+    kTrSmMaxDone = 9,   // softmax: page column maxima written (before the exchange)
+    kTrSmXchg = 10,     // softmax: exchange complete
+    kTrSmPStored = 11,  // softmax: P^T stored
+};
+struct Tracer {
+    int cta, role;
+    unsigned n;
+    bool on;
+    __device__ Tracer(int r, bool enabled = true) : cta(blockIdx.x), role(r), n(0), on(enabled) {}
+    __device__ void ev(unsigned tag) {
+        if (on && cta < kTraceCtas && n < kTraceCap)
+            g_mla_trace[cta][role][n] = (static_cast<unsigned long long>(tag) << 56) |
+                                        (global_timer_ns() & 0x00FFFFFFFFFFFFFFull);
+        ++n;
+    }
+    __device__ ~Tracer() {
+        if (on && cta < kTraceCtas) g_mla_trace_count[cta][role] = n;
+    }
+};
+#define MLA_TRACE_DECL(role) Tracer tracer_(role)
+#define MLA_TRACE_EV(tag) tracer_.ev(tag)
+#else
+#define MLA_TRACE_DECL(role)
+#define MLA_TRACE_EV(tag)
+#endif
 
 struct FwdParams {
     const int32_t* sched;
     const int32_t* block_table;
     const int32_t* seqlens;
+    const uint8_t* kv;  // page pool base (for L2 prefetch)
     __nv_bfloat16* out;
     float* lse;
     float* opart;  // [slots][NG][512]
@@ -85,14 +155,18 @@ struct FwdSmem {
     static constexpr int kRedOff = kPOff + 2 * kPBytes;       // float [2][NG][4] page maxima
     static constexpr int kSumOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]   row sums
     static constexpr int kBarOff = kSumOff + NG * 4 * 4;
-    static constexpr int kNumBars = 20;
+    static constexpr int kNumBars = 24;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KB
-    static constexpr int kTmemCols = NG == 16 ? 128 : 256;    // 2 S^T buffers + O^T (4 chunks)
-    static constexpr int kSCol = 0;                           // S^T buffer i at column i*NG
-    static constexpr int kOCol = 2 * NG;                      // O^T chunk c at column kOCol + c*NG
-    static_assert(6 * NG <= kTmemCols, "TMEM budget");
+    // TMEM columns: S^T buffer i, chain c at kSCol + (i*kSChains + c)*NG;
+    // O^T d_v chunk c at kOCol + c*NG.
+    static constexpr int kSCol = 0;
+    static constexpr int kOCol = 2 * kSChains * NG;
+    static constexpr int kTmemUsed = kOCol + 4 * NG;
+    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                   : kTmemUsed <= 256 ? 256 : 512;
+    static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0, "swizzle atoms need 1 KB alignment");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
@@ -100,7 +174,7 @@ struct FwdSmem {
 enum Bar {
     kKvFull0 = 0, kKvFull1, kKvEmpty0, kKvEmpty1, kQFull, kQEmpty,
     kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
-    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kBarCount
+    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kBarCount
 };
 
 // ------------------------------------------------------------------ waits
@@ -263,7 +337,9 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     Item item;
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
+    MLA_TRACE_DECL(0);
     while (ok && it.next(p, bginfo, item)) {
+        MLA_TRACE_EV(kTrItem);
         ok = wait_bounded(bar0 + 8 * kQEmpty, (q_it & 1) ^ 1, ctl);
         if (!ok) break;
         mbar_arrive_expect_tx(bar0 + 8 * kQFull, L::kQBytes);
@@ -273,10 +349,23 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
             tma_load_2d(q_s + c * L::kQBoxBytes, q_map, bar0 + 8 * kQFull, c * L::kBoxCols, row0);
         ++q_it;
         const int32_t* bt = p.block_table + (size_t)item.b * p.max_blocks;
+        const bool prefetch = kPrefetchPages > 0 && item.p1 - item.p0 >= kPrefetchMinPages;
+        if (prefetch)
+            for (int j = item.p0; j < item.p1 && j < item.p0 + kPrefetchPages; ++j) {
+                const int ph = __ldg(bt + j);
+                if ((unsigned)ph < (unsigned)p.num_blocks)
+                    prefetch_l2_bulk(p.kv + (size_t)ph * L::kStageBytes, L::kStageBytes);
+            }
         for (int j = item.p0; j < item.p1; ++j) {
+            if (prefetch && j + kPrefetchPages < item.p1) {
+                const int ph = __ldg(bt + j + kPrefetchPages);
+                if ((unsigned)ph < (unsigned)p.num_blocks)
+                    prefetch_l2_bulk(p.kv + (size_t)ph * L::kStageBytes, L::kStageBytes);
+            }
             const int st = kv_it & 1;
             ok = wait_bounded(bar0 + 8 * (kKvEmpty0 + st), ((kv_it >> 1) & 1) ^ 1, ctl);
             if (!ok) break;
+            MLA_TRACE_EV(kTrProdIssue);
             int phys = __ldg(bt + j);
             if ((unsigned)phys >= (unsigned)p.num_blocks) {
                 atomicOr(p.status, MLA_STATUS_BAD_BLOCK_TABLE);
@@ -301,101 +390,126 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     }
 }
 
+// GEMM1 issuer: S^T[64 x NG] = K[64 x 576] . Q^T as soon as a page has landed
+// and its S^T buffer is free.  K-major A (64 token rows of 128 B per box,
+// 8-row groups 1 KB apart) and K-major B (Q^T rows); the 16-wide k-step
+// advances 32 B inside the 128-byte swizzle atom.  k-step i accumulates into
+// the accumulator of its issuer.
 template <int NG>
-__device__ void run_mma(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
-                        uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
+__device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                          uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
     using L = FwdSmem<NG>;
-    constexpr uint32_t kIdescS = idesc_bf16_f32(64, NG, 0, 0);   // S^T = K . Q^T
-    constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);  // O^T += V^T . P^T
-    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : kSwizzle64;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(64, NG, 0, 0);
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t q_s = smem_addr(smem + L::kQOff);
+    const uint32_t bar0 = smem_addr(smem + L::kBarOff);
+    WorkIter it;
+    it.init(meta);
+    Item item;
+    uint32_t s_it = 0, q_it = 0;
+    bool ok = true, issued = false;
+#ifdef MLA_TRACE
+    Tracer tracer_(issuer == 0 ? 1 : 0, issuer == 0);
+#endif
+    // Descriptors differ only in their start address (bits 0..13, in 16-byte
+    // units): build them once and add offsets.
+    const uint64_t a_desc0 = smem_desc(kv_s, 16, 1024, kSwizzle128);
+    const uint64_t b_desc0 = smem_desc(q_s, 16, 1024, kSwizzle128);
+    while (ok && it.next(p, bginfo, item)) {
+        ok = wait_bounded(bar0 + 8 * kQFull, q_it & 1, ctl);
+        if (!ok) break;
+        for (int j = item.p0; j < item.p1; ++j) {
+            const int st = s_it & 1;
+            const uint32_t par = (s_it >> 1) & 1;
+            ok = wait_bounded(bar0 + 8 * (kKvFull0 + st), par, ctl);
+            if (!ok) break;
+            MLA_TRACE_EV(kTrMmaKvFull);
+            ok = wait_bounded(bar0 + 8 * (kSEmpty0 + st), par ^ 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            // This issuer's accumulator; it takes boxes issuer, issuer + 2, ...
+            const uint32_t d = tmem + L::kSCol + (st * kSChains + issuer) * NG;
+            const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
+            bool first = true;
+#pragma unroll 1
+            for (int c = issuer; c < L::kBoxes; c += kG1Issuers) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t a = a_st + ((c * L::kBoxBytes + k * 32) >> 4);
+                    const uint64_t b = b_desc0 + ((c * L::kQBoxBytes + k * 32) >> 4);
+                    umma_f16(d, a, b, kIdescS, first ? 0u : 1u);
+                    first = false;
+                }
+            }
+            issued = true;
+            umma_commit(bar0 + 8 * (kSFull0 + st));
+            if (j == item.p1 - 1) umma_commit(bar0 + 8 * kQEmpty);
+            ++s_it;
+        }
+        ++q_it;
+    }
+    if (issued) {
+        umma_commit(bar0 + 8 * kMmaDone);
+        wait_drain(bar0 + 8 * kMmaDone, 0);
+    }
+}
+
+// GEMM2 issuer: O^T[512 x NG] += V^T[512 x 64] . P^T as soon as P^T is in
+// shared memory.  V^T is the stage's first 8 boxes read MN-major (d_v
+// contiguous within a token row; 64 d_v per swizzle atom, next atom = next box
+// 8 KB on, 8-token groups 1 KB apart); P^T is MN-major with NG columns per
+// token row.  k-outer order keeps consecutive MMAs on different accumulators.
+template <int NG>
+__device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                          uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
+    using L = FwdSmem<NG>;
+    constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
+    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : kSwizzle64;
+    const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t p_s = smem_addr(smem + L::kPOff);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     WorkIter it;
     it.init(meta);
     Item item;
-    uint32_t kv_it = 0, s_it = 0, q_it = 0, item_it = 0;
+    uint32_t s_it = 0, item_it = 0;
     bool ok = true, issued = false;
-
-    // GEMM2 of one page: reads the V columns of stage `st` (MN-major: d_v is
-    // contiguous within a token row; 64 d_v per swizzle atom, next atom = next
-    // box, 8-token groups 1 KB apart) and P^T buffer (sidx & 1) (MN-major:
-    // NG columns contiguous per token row).
-    auto gemm2 = [&](int st, uint32_t sidx, bool first) -> bool {
-        const int pb = sidx & 1;
-        if (!wait_bounded(bar0 + 8 * (kPFull0 + pb), (sidx >> 1) & 1, ctl)) return false;
-        if (first && !wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl)) return false;
-        tc_fence_after();
-        const uint32_t a0 = kv_s + st * L::kStageBytes;
-        const uint32_t b0 = p_s + pb * L::kPBytes;
-#pragma unroll
-        for (int ch = 0; ch < kDv / 128; ++ch) {
-            const uint32_t d = tmem + L::kOCol + ch * NG;
+    MLA_TRACE_DECL(2);
+    const uint64_t a_desc0 = smem_desc(kv_s, L::kBoxBytes, 1024, kSwizzle128);
+    const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NG * 2, kPSwizzle);
+    while (ok && it.next(p, bginfo, item)) {
+        for (int j = item.p0; j < item.p1; ++j) {
+            const int st = s_it & 1;
+            const bool first = (j == item.p0);
+            ok = wait_bounded(bar0 + 8 * (kPFull0 + st), (s_it >> 1) & 1, ctl);
+            if (!ok) break;
+            if (first) {
+                ok = wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl);
+                if (!ok) break;
+            }
+            MLA_TRACE_EV(kTrMmaPFull);
+            tc_fence_after();
+            const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
+            const uint64_t b_st = b_desc0 + ((st * L::kPBytes) >> 4);
 #pragma unroll
             for (int k = 0; k < kPage / 16; ++k) {
-                const uint64_t a = smem_desc(a0 + (2 * ch) * L::kBoxBytes + k * 2048, L::kBoxBytes, 1024,
-                                             kSwizzle128);
-                const uint64_t b = smem_desc(b0 + k * 16 * NG * 2, L::kPBytes, 8 * NG * 2, kPSwizzle);
-                umma_f16(d, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
-            }
-        }
-        umma_commit(bar0 + 8 * (kKvEmpty0 + st));
-        umma_commit(bar0 + 8 * (kPEmpty0 + pb));
-        return true;
-    };
-
-    while (ok && it.next(p, bginfo, item)) {
-        ok = wait_bounded(bar0 + 8 * kQFull, q_it & 1, ctl);
-        if (!ok) break;
-        const int npages = item.p1 - item.p0;
-        int pend_st = -1;
-        uint32_t pend_s = 0;
-        bool pend_first = false;
-        for (int jj = 0; jj < npages; ++jj) {
-            const int st = kv_it & 1;
-            ok = wait_bounded(bar0 + 8 * (kKvFull0 + st), (kv_it >> 1) & 1, ctl);
-            if (!ok) break;
-            const int sb = s_it & 1;
-            ok = wait_bounded(bar0 + 8 * (kSEmpty0 + sb), ((s_it >> 1) & 1) ^ 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            // GEMM1: K-major A (64 token rows of 128 B per box, 8-row groups 1 KB
-            // apart) and K-major B (Q^T rows); the 16-wide k-step advances 32 B
-            // inside the 128-byte swizzle atom.
-            const uint32_t d = tmem + L::kSCol + sb * NG;
-            const uint32_t a0 = kv_s + st * L::kStageBytes;
-#pragma unroll 1
-            for (int c = 0; c < L::kBoxes; ++c) {
+                const uint64_t b = b_st + ((k * 16 * NG * 2) >> 4);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t a = smem_desc(a0 + c * L::kBoxBytes + k * 32, 16, 1024, kSwizzle128);
-                    const uint64_t b = smem_desc(q_s + c * L::kQBoxBytes + k * 32, 16, 1024, kSwizzle128);
-                    umma_f16(d, a, b, kIdescS, (c | k) ? 1u : 0u);
+                for (int ch = 0; ch < kDv / 128; ++ch) {
+                    const uint64_t a = a_st + (((2 * ch) * L::kBoxBytes + k * 2048) >> 4);
+                    umma_f16(tmem + L::kOCol + ch * NG, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
                 }
             }
             issued = true;
-            umma_commit(bar0 + 8 * (kSFull0 + sb));
-            if (jj == npages - 1) umma_commit(bar0 + 8 * kQEmpty);
-            if (pend_st >= 0) {
-                ok = gemm2(pend_st, pend_s, pend_first);
-                if (!ok) break;
-            }
-            pend_st = st;
-            pend_s = s_it;
-            pend_first = (jj == 0);
-            ++kv_it;
+            umma_commit(bar0 + 8 * (kKvEmpty0 + st));
+            umma_commit(bar0 + 8 * (kPEmpty0 + st));
             ++s_it;
         }
         if (!ok) break;
-        ok = gemm2(pend_st, pend_s, pend_first);
-        if (!ok) break;
-        ++q_it;
         ++item_it;
     }
     if (issued) {
-        umma_commit(bar0 + 8 * kMmaDone);
-        wait_drain(bar0 + 8 * kMmaDone, 0);
+        umma_commit(bar0 + 8 * kMmaDone2);
+        wait_drain(bar0 + 8 * kMmaDone2, 0);
     }
 }
 
@@ -407,7 +521,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     const int lane = threadIdx.x & 31;
     const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const int gt = threadIdx.x - 64;                      // 0..127 within the softmax group
+    const int gt = threadIdx.x - 128;                     // 0..127 within the softmax group
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
     float* sred = reinterpret_cast<float*>(smem + L::kSumOff);
@@ -423,6 +537,14 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     Item item;
     uint32_t s_it = 0, item_it = 0;
     bool ok = true;
+#ifdef MLA_TRACE
+    Tracer tracer_(3);
+    const bool tr = (gt == 0);
+#define MLA_TRACE_SM(tag) \
+    if (tr) tracer_.ev(tag)
+#else
+#define MLA_TRACE_SM(tag)
+#endif
     while (ok && it.next(p, bginfo, item)) {
         int lvis[NG];
 #pragma unroll
@@ -445,10 +567,20 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             const int sb = s_it & 1;
             ok = wait_warp(bar0 + 8 * (kSFull0 + sb), (s_it >> 1) & 1, ctl);
             if (!ok) break;
+            MLA_TRACE_SM(kTrSmSFull);
             tc_fence_after();
             float x[NG];
-            tmem_load_cols<NG>(tmem + lane_base + L::kSCol + sb * NG, x);
+            const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG;
+            tmem_load_cols<NG>(sbase, x);
             tmem_ld_wait();
+#pragma unroll
+            for (int c = 1; c < kSChains; ++c) {
+                float y[NG];
+                tmem_load_cols<NG>(sbase + c * NG, y);
+                tmem_ld_wait();
+#pragma unroll
+                for (int n = 0; n < NG; ++n) x[n] += y[n];
+            }
             tc_fence_before();
             mbar_arrive(bar0 + 8 * (kSEmpty0 + sb));
 
@@ -458,15 +590,19 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 
             // Column maxima of this page: warp transpose-reduce, then the four
             // warps meet through shared memory.
-            float xr[NG];
-#pragma unroll
-            for (int n = 0; n < NG; ++n) xr[n] = x[n];
-            const float wmax = ColReduce<NG, 16, true>::run(xr, lane);
             float* rb = red + (s_it & 1) * NG * 4;
-            if (reduced_writer<NG>(lane)) rb[reduced_col<NG>(lane) * 4 + wq] = wmax;
+            {
+                float xr[NG];
+#pragma unroll
+                for (int n = 0; n < NG; ++n) xr[n] = x[n];
+                const float wmax = ColReduce<NG, 16, true>::run(xr, lane);
+                if (reduced_writer<NG>(lane)) rb[reduced_col<NG>(lane) * 4 + wq] = wmax;
+            }
+            MLA_TRACE_SM(kTrSmMaxDone);
             mbar_arrive(bar0 + 8 * (kRedFull0 + (s_it & 1)));
             ok = wait_warp(bar0 + 8 * (kRedFull0 + (s_it & 1)), (s_it >> 1) & 1, ctl);
             if (!ok) break;
+            MLA_TRACE_SM(kTrSmXchg);
 
             float alpha[NG];
             bool rescale = false;
@@ -510,6 +646,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 }
             }
             fence_proxy_async_smem();
+            MLA_TRACE_SM(kTrSmPStored);
             if (rescale && j > item.p0) {
                 // O^T already holds earlier pages: wait for the previous GEMM2,
                 // then scale each column by its alpha in place.
@@ -530,6 +667,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 tmem_st_wait();
             }
             tc_fence_before();
+            MLA_TRACE_SM(kTrSmPDone);
             mbar_arrive(bar0 + 8 * (kPFull0 + pb));
             ++s_it;
         }
@@ -539,6 +677,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         const uint32_t last = s_it - 1;
         ok = wait_warp(bar0 + 8 * (kPEmpty0 + (last & 1)), (last >> 1) & 1, ctl);
         if (!ok) break;
+        MLA_TRACE_SM(kTrSmEpi0);
         tc_fence_after();
         float lr[NG];
 #pragma unroll
@@ -593,6 +732,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             }
         }
         if (!item.unsplit && item.slot < 0 && gt == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        MLA_TRACE_SM(kTrSmEpi1);
         tc_fence_before();
         mbar_arrive(bar0 + 8 * kOEmpty);
         ++item_it;
@@ -628,6 +768,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
                 i == kRedFull0 || i == kRedFull1 || i == kSumFull)
                 count = 128;
+            if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = kG1Issuers;
             mbar_init(bar0 + 8 * i, count);
         }
         *abort_flag = 0;
@@ -649,8 +790,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             prefetch_tensormap(&q_map);
             run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
         }
-    } else if (warp == 1) {
-        if (lane == 0) run_mma<NG>(p, meta, bginfo, smem, tmem, ctl);
+    } else if (warp <= kG1Issuers) {
+        if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
+    } else if (warp == kG1Issuers + 1) {
+        if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl);
     } else {
         run_softmax<NG>(p, meta, bginfo, smem, tmem, ctl);
     }
@@ -662,15 +805,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
 }
 
-// LSE-weighted merge of split partials; one CTA per (request, head group).
+// LSE-weighted merge of split partials; one CTA per (request-group, column).
 __global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombineParams p) {
     const int bg = blockIdx.x;
+    const int n = blockIdx.y;
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
         __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != p.NG) {
-        if (threadIdx.x == 0 && bg == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+        if (threadIdx.x == 0 && bg == 0 && n == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
+    const int b = bg / p.Hg;
+    const int g = bg - b * p.Hg;
+    const int gc = g * p.NG + n;
+    if (gc >= p.N) return;
     const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
     const int base = __ldg(info + 0);
     const int k = __ldg(info + 1);
@@ -679,42 +827,37 @@ __global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombinePa
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
-    const int b = bg / p.Hg;
-    const int g = bg - b * p.Hg;
+    const int s = gc / p.heads;
+    const int head = gc - s * p.heads;
     const int d0 = threadIdx.x * 4;
-    for (int n = 0; n < p.NG; ++n) {
-        const int gc = g * p.NG + n;
-        if (gc >= p.N) break;
-        const int s = gc / p.heads;
-        const int head = gc - s * p.heads;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float lstar = -INFINITY;
-        if (k > 1) {
-            float mx = -INFINITY;
-            for (int i = 0; i < k; ++i) mx = fmaxf(mx, __ldg(p.lpart + (size_t)(base + i) * p.NG + n));
-            if (mx != -INFINITY) {
-                float sum = 0.f;
-                for (int i = 0; i < k; ++i) sum += expf(__ldg(p.lpart + (size_t)(base + i) * p.NG + n) - mx);
-                lstar = mx + logf(sum);
-                for (int i = 0; i < k; ++i) {
-                    const float w = expf(__ldg(p.lpart + (size_t)(base + i) * p.NG + n) - lstar);
-                    const float4 v = __ldg(reinterpret_cast<const float4*>(
-                        p.opart + ((size_t)(base + i) * p.NG + n) * kDv + d0));
-                    acc.x += w * v.x;
-                    acc.y += w * v.y;
-                    acc.z += w * v.z;
-                    acc.w += w * v.w;
-                }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lstar = -INFINITY;
+    if (k > 1) {
+        const float* lp = p.lpart + (size_t)base * p.NG + n;
+        float mx = -INFINITY;
+        for (int i = 0; i < k; ++i) mx = fmaxf(mx, __ldg(lp + (size_t)i * p.NG));
+        if (mx != -INFINITY) {
+            float sum = 0.f;
+            for (int i = 0; i < k; ++i) sum += expf(__ldg(lp + (size_t)i * p.NG) - mx);
+            lstar = mx + logf(sum);
+            const float* op = p.opart + ((size_t)base * p.NG + n) * kDv + d0;
+            for (int i = 0; i < k; ++i) {
+                const float w = expf(__ldg(lp + (size_t)i * p.NG) - lstar);
+                const float4 v = __ldg(reinterpret_cast<const float4*>(op + (size_t)i * p.NG * kDv));
+                acc.x += w * v.x;
+                acc.y += w * v.y;
+                acc.z += w * v.z;
+                acc.w += w * v.w;
             }
         }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 packed;
-        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(p.out + (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0) = packed;
-        if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
     }
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p.out + (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0) = packed;
+    if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
 }
 
 // Block-wide inclusive scan of one int per thread (blockDim.x == 1024).
@@ -743,19 +886,30 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
 }
 
 // Builds the persistent-CTA plan on the device (one block of 1024 threads).
+// With use_smem the lengths and the unit prefix live in dynamic shared memory
+// ((B + BG + 1) int32), so the per-CTA binary searches stay on chip; the
+// prefix is also written to the schedule buffer.
 __global__ void __launch_bounds__(1024)
-    mla_decode_schedule_kernel(const int32_t* __restrict__ seqlens, int32_t* __restrict__ sched, int B,
-                               int Hg, int NG, int G, int max_blocks) {
+    mla_decode_schedule_kernel(const int32_t* __restrict__ seqlens_g, int32_t* __restrict__ sched, int B,
+                               int Hg, int NG, int G, int max_blocks, int use_smem) {
+    extern __shared__ int32_t sh[];
     __shared__ int warp_tot[32];
     __shared__ int carry;
     __shared__ int bad_len;
     const int BG = B * Hg;
-    int32_t* prefix = sched + prefix_offset_words(G, BG);
+    int32_t* prefix_g = sched + prefix_offset_words(G, BG);
     int32_t* bginfo = sched + bg_offset_words(G);
     int32_t* meta = sched + kHdrWords;
+    const int32_t* seqlens = seqlens_g;
+    int32_t* prefix = prefix_g;
     if (threadIdx.x == 0) {
         carry = 0;
         bad_len = 0;
+    }
+    if (use_smem) {
+        for (int i = threadIdx.x; i < B; i += 1024) sh[i] = seqlens_g[i];
+        seqlens = sh;
+        prefix = sh + B;
     }
     __syncthreads();
     for (int base = 0; base < BG; base += 1024) {
@@ -767,13 +921,19 @@ __global__ void __launch_bounds__(1024)
             v = (int)units_of(pages_of(clamp_seqlen(L, max_blocks)));
         }
         const int incl = block_inclusive_scan(v, warp_tot);
-        if (bg < BG) prefix[bg] = carry + incl - v;
+        if (bg < BG) {
+            prefix[bg] = carry + incl - v;
+            if (use_smem) prefix_g[bg] = carry + incl - v;
+        }
         __syncthreads();
         if (threadIdx.x == 1023) carry += incl;
         __syncthreads();
     }
     const int64_t W = carry;
-    if (threadIdx.x == 0) prefix[BG] = (int)W;
+    if (threadIdx.x == 0) {
+        prefix[BG] = (int)W;
+        prefix_g[BG] = (int)W;
+    }
     __syncthreads();
     const int64_t T = units_per_cta(W, G);
     for (int k = threadIdx.x; k < G; k += 1024)

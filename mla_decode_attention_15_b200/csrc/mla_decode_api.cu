@@ -166,7 +166,7 @@ int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedul
     c.G = pl.G;
     c.BG = pl.BG;
     c.slots_cap = (int)pl.slots;
-    mla_decode_combine_kernel<<<pl.BG, 128, 0, stream>>>(c);
+    mla_decode_combine_kernel<<<dim3(pl.BG, pl.gr.NG), 128, 0, stream>>>(c);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -205,9 +205,12 @@ int mla_decode_get_schedule(const mla_decode_dims* dims, const int32_t* cache_se
     int rc = make_plan(dims, &pl);
     if (rc != MLA_OK) return rc;
     if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
-    mla_decode_schedule_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+    // Lengths and unit prefix in shared memory when they fit the default 48 KB.
+    const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
+    const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
+    mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
         cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.gr.Hg, pl.gr.NG, pl.G,
-        dims->max_blocks_per_seq);
+        dims->max_blocks_per_seq, use_smem);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -272,6 +275,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.sched = static_cast<const int32_t*>(schedule);
     p.block_table = block_table;
     p.seqlens = cache_seqlens;
+    p.kv = static_cast<const uint8_t*>(kv_cache);
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
     p.opart = static_cast<float*>(workspace);
@@ -304,6 +308,20 @@ int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const 
         return MLA_ERR_INVALID_ARG;
     return launch_combine(dims, pl, schedule, workspace, out, lse, static_cast<cudaStream_t>(stream));
 }
+
+#ifdef MLA_TRACE
+// Tracing builds only: copies the per-CTA event buffer (see decode_kernels.cuh)
+// and the per-role event counts to host memory.
+int mla_decode_trace_fetch(void* events_host, size_t events_bytes, void* counts_host, size_t counts_bytes) {
+    if (events_bytes != sizeof(g_mla_trace) || counts_bytes != sizeof(g_mla_trace_count)) return MLA_ERR_INVALID_ARG;
+    if (cudaMemcpyFromSymbol(events_host, g_mla_trace, events_bytes) != cudaSuccess ||
+        cudaMemcpyFromSymbol(counts_host, g_mla_trace_count, counts_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+#endif
 
 int mla_decode_get_status(const void* schedule, int32_t* host_status) {
     if (!aligned16(schedule) || host_status == nullptr) return MLA_ERR_INVALID_ARG;

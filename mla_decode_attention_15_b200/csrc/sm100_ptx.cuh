@@ -66,6 +66,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     return pol;
 }
 
+// Bulk prefetch of a contiguous global range into L2 (no shared memory involved).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gptr)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint32_t bar, int c0,
                                             int c1) {
     asm volatile(
