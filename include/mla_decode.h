@@ -60,6 +60,7 @@ extern "C" {
 #define MLA_ERR_UNSUPPORTED (-2)  /* page_size != 64, d_qk != 576, d_v != 512, heads*s_q > 256 */
 #define MLA_ERR_CUDA (-3)         /* a CUDA runtime/driver call or launch failed */
 #define MLA_ERR_BAD_SCHEDULE (-4) /* schedule buffer was not built for these dims */
+#define MLA_ERR_SCRATCH_TOO_SMALL (-5) /* mla_decode_fwd_noalloc: the request needs more than its built-in scratch */
 
 /* device status bits (mla_decode_get_status) */
 #define MLA_STATUS_BAD_BLOCK_TABLE 0x1 /* an entry was outside [0, num_blocks); page 0 was read instead */
@@ -144,6 +145,35 @@ int mla_decode_get_status(const void* schedule, int32_t* host_status);
 
 /* Static text for an MLA_* return code. */
 const char* mla_decode_strerror(int code);
+
+/* Allocation-free decode: schedule + decode + combine in one call, for callers
+ * that cannot allocate device memory themselves -- for example a runtime or
+ * plugin host that plans every device buffer ahead of time and gives a kernel
+ * library no allocator, or a decode loop that cannot afford cudaMalloc's
+ * implicit device synchronisation.  The pages describe no such entry point;
+ * it exists for the library's users only.
+ *
+ * Arguments and results are those of mla_decode_fwd (dims->flags must not
+ * contain MLA_FLAG_NO_COMBINE).  Instead of caller-provided schedule and
+ * workspace buffers it uses one scratch array of MLA_NOALLOC_SCRATCH_BYTES
+ * that the library declares in device memory; every GPU that loads the
+ * library holds that array until the process exits.  Requests whose schedule
+ * plus split partials would exceed it return MLA_ERR_SCRATCH_TOO_SMALL before
+ * anything is enqueued; use mla_decode_fwd then.
+ *   - No call allocates or frees device or host memory.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, cached per device); make that first call before
+ *     any stream capture on that device.
+ *   - All calls share the one array, and it keeps the previous call's
+ *     contents (the schedule kernel rewrites the parts that must start fresh).
+ *     Calls whose GPU work overlaps -- different streams without ordering,
+ *     or several threads at once -- race on it and give wrong results;
+ *     serialise them.
+ *   - The device status word lives in the array and is not reported. */
+#define MLA_NOALLOC_SCRATCH_BYTES (24u << 20)
+int mla_decode_fwd_noalloc(const mla_decode_dims* dims, const void* q, const void* kv_cache,
+                           const int32_t* block_table, const int32_t* cache_seqlens,
+                           float softmax_scale, void* out, float* lse, void* stream);
 
 /* Library ABI version (increments on any change of these declarations). */
 int mla_decode_version(void);

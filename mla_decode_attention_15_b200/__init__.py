@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     mla_decode,
     mla_decode_combine,
     mla_decode_fwd,
+    mla_decode_fwd_noalloc,
     mla_decode_get_schedule,
     mla_decode_get_schedule_host,
     mla_decode_get_status,

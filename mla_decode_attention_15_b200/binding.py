@@ -20,6 +20,8 @@ MLA_ERR_INVALID_ARG = -1
 MLA_ERR_UNSUPPORTED = -2
 MLA_ERR_CUDA = -3
 MLA_ERR_BAD_SCHEDULE = -4
+MLA_ERR_SCRATCH_TOO_SMALL = -5
+MLA_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 MLA_STATUS_BAD_BLOCK_TABLE = 0x1
 MLA_STATUS_TIMEOUT = 0x2
@@ -38,6 +40,7 @@ EXPORTED = (
     "mla_decode_get_schedule",
     "mla_decode_get_schedule_host",
     "mla_decode_fwd",
+    "mla_decode_fwd_noalloc",
     "mla_decode_combine",
     "mla_decode_get_status",
     "mla_decode_strerror",
@@ -84,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_get_schedule_host.argtypes = [P, vp, vp]
         L.mla_decode_fwd.restype = ctypes.c_int
         L.mla_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+        L.mla_decode_fwd_noalloc.restype = ctypes.c_int
+        L.mla_decode_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
         L.mla_decode_combine.restype = ctypes.c_int
         L.mla_decode_combine.argtypes = [P, vp, vp, vp, vp, vp]
         L.mla_decode_get_status.restype = ctypes.c_int
@@ -153,6 +158,17 @@ def mla_decode_fwd(dims, schedule, workspace, q, kv_cache, block_table, cache_se
                                 _ptr(kv_cache), _ptr(block_table), _ptr(cache_seqlens),
                                 float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)),
            "mla_decode_fwd")
+
+
+def mla_decode_fwd_noalloc(dims, q, kv_cache, block_table, cache_seqlens, softmax_scale: float,
+                           out, lse, stream=None) -> None:
+    """Schedule + decode + combine without caller-provided schedule or
+    workspace: the library uses its own fixed device scratch (see the header).
+    For callers that cannot allocate device memory.  Calls that overlap on the
+    GPU share that scratch and race; serialise them."""
+    _check(lib().mla_decode_fwd_noalloc(ctypes.byref(dims), _ptr(q), _ptr(kv_cache), _ptr(block_table),
+                                        _ptr(cache_seqlens), float(softmax_scale), _ptr(out), _ptr(lse),
+                                        _stream(stream)), "mla_decode_fwd_noalloc")
 
 
 def mla_decode_combine(dims, schedule, workspace, out, lse, stream=None) -> None:

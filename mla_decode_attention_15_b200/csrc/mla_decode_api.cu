@@ -170,6 +170,36 @@ int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedul
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// ---- scratch of the allocation-free entry point ----
+// One array per device, in this library's module; allocated by the driver when
+// the module is loaded on a device and held until the process exits.
+constexpr size_t kNoAllocScratchBytes = MLA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_mla_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch on the current device.  In host code the
+// array's name is only a host-side handle, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+    static void* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_mla_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+        addr[dev] = ptr;
+    }
+    *out = addr[dev];
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -183,6 +213,9 @@ const char* mla_decode_strerror(int code) {
         case MLA_ERR_UNSUPPORTED: return "unsupported shape (page_size must be 64, d_qk 576, d_v 512, heads*s_q <= 256)";
         case MLA_ERR_CUDA: return "CUDA runtime or launch error";
         case MLA_ERR_BAD_SCHEDULE: return "schedule buffer does not match these dims";
+        case MLA_ERR_SCRATCH_TOO_SMALL:
+            return "request needs more than the 24 MiB built-in scratch of mla_decode_fwd_noalloc; "
+                   "use mla_decode_fwd with caller-allocated schedule and workspace";
         default: return "unknown error code";
     }
 }
@@ -322,6 +355,30 @@ int mla_decode_trace_fetch(void* events_host, size_t events_bytes, void* counts_
     return MLA_OK;
 }
 #endif
+
+int mla_decode_fwd_noalloc(const mla_decode_dims* dims, const void* q, const void* kv_cache,
+                           const int32_t* block_table, const int32_t* cache_seqlens, float softmax_scale,
+                           void* out, float* lse, void* stream) {
+    Plan pl;
+    int rc = make_plan(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_ERR_INVALID_ARG;  // no workspace to combine from later
+    if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(block_table) || !aligned16(cache_seqlens) ||
+        !aligned16(out) || !aligned16(lse) || !std::isfinite(softmax_scale))
+        return MLA_ERR_INVALID_ARG;
+    const size_t sched_bytes = ((size_t)schedule_words(pl.G, pl.BG) * sizeof(int32_t) + 255) & ~(size_t)255;
+    const size_t ws_bytes = workspace_bytes_of(pl);
+    if (sched_bytes + ws_bytes > kNoAllocScratchBytes) return MLA_ERR_SCRATCH_TOO_SMALL;
+    void* base = nullptr;
+    rc = noalloc_scratch(&base);
+    if (rc != MLA_OK) return rc;
+    uint8_t* schedule = static_cast<uint8_t*>(base);
+    uint8_t* workspace = schedule + sched_bytes;
+    rc = mla_decode_get_schedule(dims, cache_seqlens, schedule, stream);
+    if (rc != MLA_OK) return rc;
+    return mla_decode_fwd(dims, schedule, workspace, q, kv_cache, block_table, cache_seqlens, softmax_scale,
+                          out, lse, stream);
+}
 
 int mla_decode_get_status(const void* schedule, int32_t* host_status) {
     if (!aligned16(schedule) || host_status == nullptr) return MLA_ERR_INVALID_ARG;
