@@ -189,6 +189,20 @@ def rank_seed(base_seed: int, rank: int) -> int:
     return base_seed + 7919 * rank
 
 
+def aggregate_over_ranks(times_ms, kv_bytes: float, device) -> tuple:
+    """Whole-job view of a weak-scaling run: every time is the slowest rank's
+    (MAX over ranks), the KV bytes are summed over ranks.  Single process:
+    returned unchanged."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(times_ms), float(kv_bytes)
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    b = torch.tensor([float(kv_bytes)], dtype=torch.float64, device=device)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()], float(b[0])
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample_rate(d, w, budget_s: float, max_requests=None):
     """Times the fp64 oracle on whole requests (all heads x s_q rows of each)
@@ -342,16 +356,7 @@ def run_ours(args, w):
     status = bd.mla_decode_get_status(sched)
     assert status == 0, "device status %#x" % status
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_step, kernel_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, kernel_ms = float(t[0]), float(t[1])
-        tot = torch.tensor([byt["kv"]], dtype=torch.float64, device=dev)
-        dist.all_reduce(tot)
-        total_kv = float(tot[0])
-    else:
-        total_kv = float(byt["kv"])
+    (ms_step, kernel_ms), total_kv = aggregate_over_ranks([ms_step, kernel_ms], byt["kv"], dev)
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -441,12 +446,7 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
-    kvb = algorithmic_bytes(d["cache_seqlens"], s_q, h)["kv"] * world
+    (ms,), kvb = aggregate_over_ranks([ms], algorithmic_bytes(d["cache_seqlens"], s_q, h)["kv"], dev)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     return {"value": kvb / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,

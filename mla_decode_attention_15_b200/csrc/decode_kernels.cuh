@@ -197,7 +197,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
     }
 }
 
-// All 32 lanes wait; the verdict is made warp-uniform so that the warp keeps
+// All 32 lanes wait; the outcome is made warp-uniform so that the warp keeps
 // executing .sync.aligned instructions together.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& c) {
     const bool ok = wait_bounded(bar, parity, c);

@@ -27,7 +27,7 @@
  *    The full row (latent + RoPE key) is the key; the latent (the first d_v
  *    columns) is the value.
  *  - FlashMLA-ETAP technical summary, "Estabilidade Numérica": accuracy is
- *    judged against a double-precision reference, which this is.
+ *    measured against a double-precision reference, which this is.
  *
  * Readings where the pages are silent (each is also listed in the design
  * notes): the causal rule for s_q > 1 above; an empty visible range gives
