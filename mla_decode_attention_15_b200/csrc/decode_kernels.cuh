@@ -261,12 +261,25 @@ struct WorkIter {
 };
 
 // ------------------------------------------------------------------ helpers
-// Transpose-reduce across the warp: each step every lane keeps half of its
-// columns and folds in its partner's copy of them.  After it, the lane holds
-// the reduction over all 32 lanes of column (lane >> (5 - log2 W)).
-template <int W, int OFF, bool kMax>
-struct ColReduce {
+// ---- half-column layout of the softmax warps ----
+// tcgen05.ld.16x64b reads the 16 lanes of an M=64 accumulator quadrant with
+// all 32 threads.  Measured thread mapping on B200: thread t holds lane
+// (token) t/4 + 8*(t&1) and the columns of parity (t>>1)&1, one per register
+// (column parity + 2*i in register i).  So each thread owns one token and
+// half of the NG query columns ("own" columns).
+__device__ __forceinline__ int half_token(int lane) { return (lane >> 2) + 8 * (lane & 1); }
+__device__ __forceinline__ int half_parity(int lane) { return (lane >> 1) & 1; }
+
+__host__ __device__ constexpr int half_off(int step) { return step == 0 ? 16 : step == 1 ? 8 : step == 2 ? 4 : 1; }
+
+// Transpose-reduce over the 16 threads that share a column parity (lane bits
+// 4, 3, 2 and 0; bit 1 is the parity).  Each transposing step keeps half of
+// the thread's W columns and folds in its partner's copy of them; when one
+// column is left the remaining partner bits are reduced plainly.
+template <int W, int S, bool kMax>
+struct HalfReduce {
     __device__ __forceinline__ static float run(float* v, int lane) {
+        constexpr int OFF = half_off(S);
         constexpr int H = W / 2;
         const bool upper = (lane & OFF) != 0;
 #pragma unroll
@@ -276,29 +289,55 @@ struct ColReduce {
             const float got = __shfl_xor_sync(kFullMask, send, OFF);
             v[i] = kMax ? fmaxf(keep, got) : keep + got;
         }
-        return ColReduce<H, OFF / 2, kMax>::run(v, lane);
+        return HalfReduce<H, S + 1, kMax>::run(v, lane);
     }
 };
-template <int OFF, bool kMax>
-struct ColReduce<1, OFF, kMax> {
+template <int S, bool kMax>
+struct HalfReduce<1, S, kMax> {
     __device__ __forceinline__ static float run(float* v, int) {
         float x = v[0];
 #pragma unroll
-        for (int o = OFF; o >= 1; o >>= 1) {
-            const float got = __shfl_xor_sync(kFullMask, x, o);
+        for (int s = S; s < 4; ++s) {
+            const float got = __shfl_xor_sync(kFullMask, x, half_off(s));
             x = kMax ? fmaxf(x, got) : x + got;
         }
         return x;
     }
 };
-
+// Own-column index i (column = parity + 2*i) the thread holds after HalfReduce,
+// and whether it is the one thread of its pair that writes the result.
 template <int NG>
-__device__ __forceinline__ int reduced_col(int lane) {
-    return NG == 16 ? (lane >> 1) : lane;
+__device__ __forceinline__ int half_reduced_index(int lane) {
+    return NG == 16 ? ((lane >> 2) & 7) : ((((lane >> 2) & 7) << 1) | (lane & 1));
 }
 template <int NG>
-__device__ __forceinline__ bool reduced_writer(int lane) {
+__device__ __forceinline__ bool half_reduced_writer(int lane) {
     return NG == 32 || (lane & 1) == 0;
+}
+// P^T (and so O^T) columns are stored parity-major: position q holds query
+// column 2q for q < NG/2 and column 2(q - NG/2) + 1 above.
+__host__ __device__ constexpr int pos_to_col(int q, int NG) { return q < NG / 2 ? 2 * q : 2 * (q - NG / 2) + 1; }
+
+// 16 lanes x NG/2 own columns of one accumulator (16x64b.x8 or .x16).
+template <int NG>
+__device__ __forceinline__ void tmem_load_half(uint32_t taddr, float (&v)[NG / 2]) {
+    uint32_t r[NG / 2];
+    if constexpr (NG == 16) {
+        asm volatile("tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                       "=r"(r[7])
+                     : "r"(taddr));
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.16x64b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+              "=r"(r[15])
+            : "r"(taddr));
+    }
+#pragma unroll
+    for (int i = 0; i < NG / 2; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 template <int NG>
@@ -517,6 +556,7 @@ template <int NG>
 __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                             uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
     using L = FwdSmem<NG>;
+    constexpr int W = NG / 2;                             // own columns per thread
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
@@ -526,17 +566,17 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
     float* sred = reinterpret_cast<float*>(smem + L::kSumOff);
     uint8_t* pbuf = smem + L::kPOff;
-    // In an M=64 accumulator, token row m of S^T sits in TMEM lane 32*(m/16) + m%16:
-    // lanes 0..15 of each quadrant carry 16 tokens of the page.
-    const bool row_ok = lane < 16;
-    const int row = 16 * wq + lane;
-    constexpr int kChunks = NG * 2 / 16;  // 16-byte chunks per P^T row
-
-    WorkIter it;
-    it.init(meta);
-    Item item;
-    uint32_t s_it = 0, item_it = 0;
-    bool ok = true;
+    // Token row of this thread in the page (M=64 accumulator: token m sits in
+    // TMEM lane 32*(m/16) + m%16) and its column parity.
+    const int par = half_parity(lane);
+    const int row = 16 * wq + half_token(lane);
+    const int red_i = half_reduced_index<NG>(lane);
+    const int red_col = par + 2 * red_i;
+    const bool red_w = half_reduced_writer<NG>(lane);
+    // P^T row: W bf16 at positions par*W .. par*W+W-1, in 16-byte chunks.
+    constexpr int kChunks = NG * 2 / 16;                  // 16-byte chunks per P^T row
+    constexpr int kMyChunks = kChunks / 2;
+    const int swz = ((row * NG * 2) >> 7) & (kChunks - 1);
 #ifdef MLA_TRACE
     Tracer tracer_(3);
     const bool tr = (gt == 0);
@@ -545,126 +585,160 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 #else
 #define MLA_TRACE_SM(tag)
 #endif
+
+    WorkIter it;
+    it.init(meta);
+    Item item;
+    uint32_t s_it = 0, item_it = 0;
+    bool ok = true;
     while (ok && it.next(p, bginfo, item)) {
-        int lvis[NG];
+        int lvis[W];                                      // visible length of each own column
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-            const int gc = item.g * NG + n;
+        for (int i = 0; i < W; ++i) {
+            const int gc = item.g * NG + par + 2 * i;
             int v = 0;
             if (gc < p.N) {
-                const int s = gc / p.heads;
-                v = (p.causal && p.s_q > 1) ? item.L - p.s_q + 1 + s : item.L;
+                const int sq = gc / p.heads;
+                v = (p.causal && p.s_q > 1) ? item.L - p.s_q + 1 + sq : item.L;
             }
-            lvis[n] = v;
+            lvis[i] = v;
         }
-        float m_run[NG], l_run[NG];
+        float m_all[NG];                                  // running max (log2 units), every column
+        float l_own[W];                                   // running row sum, own columns, own token
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-            m_run[n] = -INFINITY;
-            l_run[n] = 0.f;
-        }
+        for (int n = 0; n < NG; ++n) m_all[n] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < W; ++i) l_own[i] = 0.f;
+
         for (int j = item.p0; j < item.p1; ++j) {
             const int sb = s_it & 1;
             ok = wait_warp(bar0 + 8 * (kSFull0 + sb), (s_it >> 1) & 1, ctl);
             if (!ok) break;
             MLA_TRACE_SM(kTrSmSFull);
             tc_fence_after();
-            float x[NG];
-            const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG;
-            tmem_load_cols<NG>(sbase, x);
-            tmem_ld_wait();
+            float x[W];
+            {
+                const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG;
+                tmem_load_half<NG>(sbase, x);
 #pragma unroll
-            for (int c = 1; c < kSChains; ++c) {
-                float y[NG];
-                tmem_load_cols<NG>(sbase + c * NG, y);
+                for (int c = 1; c < kSChains; ++c) {
+                    float y[W];
+                    tmem_load_half<NG>(sbase + c * NG, y);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < W; ++i) x[i] += y[i];
+                }
                 tmem_ld_wait();
-#pragma unroll
-                for (int n = 0; n < NG; ++n) x[n] += y[n];
             }
             tc_fence_before();
             mbar_arrive(bar0 + 8 * (kSEmpty0 + sb));
 
             const int t = j * kPage + row;
 #pragma unroll
-            for (int n = 0; n < NG; ++n) x[n] = (row_ok && t < lvis[n]) ? x[n] * p.scale_log2 : -INFINITY;
+            for (int i = 0; i < W; ++i) x[i] = (t < lvis[i]) ? x[i] * p.scale_log2 : -INFINITY;
 
-            // Column maxima of this page: warp transpose-reduce, then the four
-            // warps meet through shared memory.
+            // Page maxima of the own columns over the 16 tokens of this warp,
+            // then the four warps meet through shared memory.
             float* rb = red + (s_it & 1) * NG * 4;
             {
-                float xr[NG];
+                float xr[W];
 #pragma unroll
-                for (int n = 0; n < NG; ++n) xr[n] = x[n];
-                const float wmax = ColReduce<NG, 16, true>::run(xr, lane);
-                if (reduced_writer<NG>(lane)) rb[reduced_col<NG>(lane) * 4 + wq] = wmax;
+                for (int i = 0; i < W; ++i) xr[i] = x[i];
+                const float wmax = HalfReduce<W, 0, true>::run(xr, lane);
+                if (red_w) rb[red_col * 4 + wq] = wmax;
             }
             MLA_TRACE_SM(kTrSmMaxDone);
             mbar_arrive(bar0 + 8 * (kRedFull0 + (s_it & 1)));
+
+            // Speculative P with the running max, stored before the exchange
+            // completes; it stands unless some column's max grows by > 2^8.
+            float m_own[W];
+#pragma unroll
+            for (int i = 0; i < W; ++i) m_own[i] = par ? m_all[2 * i + 1] : m_all[2 * i];
+            float e[W];
+#pragma unroll
+            for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
+            const int pb = s_it & 1;
+            uint8_t* rowp = pbuf + pb * L::kPBytes + row * (NG * 2);
+            auto store_p = [&](const float (&ev)[W]) {
+                uint32_t packed[W / 2];
+#pragma unroll
+                for (int i = 0; i < W; i += 2) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(ev[i], ev[i + 1]);
+                    packed[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+#pragma unroll
+                for (int c = 0; c < kMyChunks; ++c) {
+                    const int chunk = par * kMyChunks + c;
+                    *reinterpret_cast<uint4*>(rowp + ((chunk ^ swz) * 16)) =
+                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                }
+            };
+            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
+            if (!ok) break;
+            store_p(e);
+            fence_proxy_async_smem();
+            MLA_TRACE_SM(kTrSmPStored);
+
             ok = wait_warp(bar0 + 8 * (kRedFull0 + (s_it & 1)), (s_it >> 1) & 1, ctl);
             if (!ok) break;
             MLA_TRACE_SM(kTrSmXchg);
-
-            float alpha[NG];
-            bool rescale = false;
+            bool grow = false;
 #pragma unroll
-            for (int n = 0; n < NG; ++n) {
-                const float4 r4 = *reinterpret_cast<const float4*>(rb + n * 4);
+            for (int i = 0; i < W; ++i) {
+                const float4 r4 = *reinterpret_cast<const float4*>(rb + (par + 2 * i) * 4);
                 const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                const float mnew = fmaxf(m_run[n], pmax);
-                if (mnew > m_run[n] + kRescaleLog2) {
-                    alpha[n] = ex2_approx(m_run[n] - mnew);
-                    m_run[n] = mnew;
-                    rescale = true;
-                } else {
-                    alpha[n] = 1.f;
-                }
+                grow |= pmax > m_own[i] + kRescaleLog2;
             }
-            // P = 2^(x - m): GEMM2 multiplies its bf16 rounding; the row sums
-            // (and so the LSE) accumulate the fp32 values.
-            uint32_t packed[NG / 2];
+            // The warp's threads cover every column and every warp reads the
+            // same maxima, so this decision is uniform across the CTA.
+            if (!__any_sync(kFullMask, grow)) {
 #pragma unroll
-            for (int n = 0; n < NG; n += 2) {
-                const float e0 = (x[n] == -INFINITY) ? 0.f : ex2_approx(x[n] - m_run[n]);
-                const float e1 = (x[n + 1] == -INFINITY) ? 0.f : ex2_approx(x[n + 1] - m_run[n + 1]);
-                l_run[n] = l_run[n] * alpha[n] + e0;
-                l_run[n + 1] = l_run[n + 1] * alpha[n + 1] + e1;
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-                packed[n / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            const int pb = s_it & 1;
-            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
-            if (!ok) break;
-            if (row_ok) {
-                // P^T row of this token, MN-major with a (2*NG)-byte swizzle span:
-                // 16-byte chunk c of row r lands at chunk c ^ ((r*2*NG >> 7) & (kChunks-1)).
-                uint8_t* rowp = pbuf + pb * L::kPBytes + row * (NG * 2);
-                const int swz = ((row * NG * 2) >> 7) & (kChunks - 1);
+                for (int i = 0; i < W; ++i) l_own[i] += e[i];
+            } else {
+                // Slow path (first page of an item, or a jump of the max):
+                // move the reference max of the grown columns, rescale.
+                float alpha[NG];
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    *reinterpret_cast<uint4*>(rowp + ((c ^ swz) * 16)) =
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                for (int n = 0; n < NG; ++n) {
+                    const float4 r4 = *reinterpret_cast<const float4*>(rb + n * 4);
+                    const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+                    const float mnew = fmaxf(m_all[n], pmax);
+                    if (mnew > m_all[n] + kRescaleLog2) {
+                        alpha[n] = ex2_approx(m_all[n] - mnew);
+                        m_all[n] = mnew;
+                    } else {
+                        alpha[n] = 1.f;
+                    }
                 }
-            }
-            fence_proxy_async_smem();
-            MLA_TRACE_SM(kTrSmPStored);
-            if (rescale && j > item.p0) {
-                // O^T already holds earlier pages: wait for the previous GEMM2,
-                // then scale each column by its alpha in place.
-                const uint32_t prev = s_it - 1;
-                ok = wait_warp(bar0 + 8 * (kPEmpty0 + (prev & 1)), (prev >> 1) & 1, ctl);
-                if (!ok) break;
-                tc_fence_after();
+#pragma unroll
+                for (int i = 0; i < W; ++i) {
+                    const float a = par ? alpha[2 * i + 1] : alpha[2 * i];
+                    const float m = par ? m_all[2 * i + 1] : m_all[2 * i];
+                    e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m);
+                    l_own[i] = l_own[i] * a + e[i];
+                }
+                store_p(e);
+                fence_proxy_async_smem();
+                if (j > item.p0) {
+                    // O^T already holds earlier pages: wait for the previous
+                    // GEMM2, then scale each column (position) in place.
+                    const uint32_t prev = s_it - 1;
+                    ok = wait_warp(bar0 + 8 * (kPEmpty0 + (prev & 1)), (prev >> 1) & 1, ctl);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll 1
-                for (int ch = 0; ch < kDv / 128; ++ch) {
-                    float o[NG];
-                    const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
-                    tmem_load_cols<NG>(ta, o);
-                    tmem_ld_wait();
+                    for (int ch = 0; ch < kDv / 128; ++ch) {
+                        float o[NG];
+                        const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
+                        tmem_load_cols<NG>(ta, o);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int n = 0; n < NG; ++n) o[n] *= alpha[n];
-                    tmem_store_cols<NG>(ta, o);
+                        for (int q = 0; q < NG; ++q) o[q] *= alpha[pos_to_col(q, NG)];
+                        tmem_store_cols<NG>(ta, o);
+                    }
+                    tmem_st_wait();
                 }
-                tmem_st_wait();
             }
             tc_fence_before();
             MLA_TRACE_SM(kTrSmPDone);
@@ -679,11 +753,13 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         if (!ok) break;
         MLA_TRACE_SM(kTrSmEpi0);
         tc_fence_after();
-        float lr[NG];
+        {
+            float lr[W];
 #pragma unroll
-        for (int n = 0; n < NG; ++n) lr[n] = l_run[n];
-        const float wsum = ColReduce<NG, 16, false>::run(lr, lane);
-        if (reduced_writer<NG>(lane)) sred[reduced_col<NG>(lane) * 4 + wq] = wsum;
+            for (int i = 0; i < W; ++i) lr[i] = l_own[i];
+            const float wsum = HalfReduce<W, 0, false>::run(lr, lane);
+            if (red_w) sred[red_col * 4 + wq] = wsum;
+        }
         mbar_arrive(bar0 + 8 * kSumFull);
         ok = wait_warp(bar0 + 8 * kSumFull, item_it & 1, ctl);
         if (!ok) break;
@@ -701,14 +777,15 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             tmem_ld_wait();
             const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
 #pragma unroll
-            for (int n = 0; n < NG; ++n) {
+            for (int q = 0; q < NG; ++q) {
+                const int n = pos_to_col(q, NG);
                 const int gc = item.g * NG + n;
                 if (gc < p.N) {
-                    const float v = o[n] * inv[n];
+                    const float v = o[q] * inv[n];
                     if (item.unsplit) {
-                        const int s = gc / p.heads;
-                        const int head = gc - s * p.heads;
-                        p.out[(((size_t)item.b * p.s_q + s) * p.heads + head) * kDv + d] =
+                        const int sq = gc / p.heads;
+                        const int head = gc - sq * p.heads;
+                        p.out[(((size_t)item.b * p.s_q + sq) * p.heads + head) * kDv + d] =
                             __float2bfloat16_rn(v);
                     } else if (item.slot >= 0) {
                         p.opart[((size_t)item.slot * NG + n) * kDv + d] = v;
@@ -720,12 +797,12 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         for (int n = 0; n < NG; ++n) {
             const int gc = item.g * NG + n;
             if (gt == n && gc < p.N) {
-                const float lse2 = lsum[n] > 0.f ? m_run[n] + log2f(lsum[n]) : -INFINITY;
+                const float lse2 = lsum[n] > 0.f ? m_all[n] + log2f(lsum[n]) : -INFINITY;
                 const float lse = lse2 * kLn2;
                 if (item.unsplit) {
-                    const int s = gc / p.heads;
-                    const int head = gc - s * p.heads;
-                    p.lse[((size_t)item.b * p.heads + head) * p.s_q + s] = lse;
+                    const int sq = gc / p.heads;
+                    const int head = gc - sq * p.heads;
+                    p.lse[((size_t)item.b * p.heads + head) * p.s_q + sq] = lse;
                 } else if (item.slot >= 0) {
                     p.lpart[(size_t)item.slot * NG + n] = lse;
                 }
