@@ -827,6 +827,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Launched as a dependent of the schedule kernel: wait until the plan is
+    // written, then let the combine launch behind this grid.
+    griddep_wait();
+    griddep_launch_dependents();
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
         __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG) {
@@ -886,6 +890,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 __global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombineParams p) {
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
+    griddep_wait();  // the decode grid's partials are complete and visible
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
         __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != p.NG) {
@@ -973,6 +978,9 @@ __global__ void __launch_bounds__(1024)
     __shared__ int warp_tot[32];
     __shared__ int carry;
     __shared__ int bad_len;
+    // The decode kernel that follows may launch now; it waits for this grid
+    // to complete before it reads the plan.
+    griddep_launch_dependents();
     const int BG = B * Hg;
     int32_t* prefix_g = sched + prefix_offset_words(G, BG);
     int32_t* bginfo = sched + bg_offset_words(G);

@@ -145,7 +145,20 @@ int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const
                cudaStream_t stream) {
     int rc = ensure_smem_attr<NG>();
     if (rc != MLA_OK) return rc;
-    mla_decode_fwd_kernel<NG><<<pl.G, kFwdThreads, FwdSmem<NG>::kAlloc, stream>>>(kvm, qm, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.G);
+    cfg.blockDim = dim3(kFwdThreads);
+    cfg.dynamicSmemBytes = FwdSmem<NG>::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla_decode_fwd_kernel<NG>, kvm, qm, p) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -166,7 +179,20 @@ int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedul
     c.G = pl.G;
     c.BG = pl.BG;
     c.slots_cap = (int)pl.slots;
-    mla_decode_combine_kernel<<<dim3(pl.BG, pl.gr.NG), 128, 0, stream>>>(c);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.BG, pl.gr.NG);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel, c) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -91,6 +91,16 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void* map, 
         : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: the next kernel in the stream may start once
+// every CTA of this one has called launch_dependents (or exited); it then
+// waits in griddep_wait until this grid has completed and its memory is
+// visible.  Both are no-ops when the launch has no such dependency.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -168,6 +168,24 @@ def test_explicit_combine_matches_fused_launch(dev):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+def test_one_plan_serves_repeated_calls(dev):
+    """One plan serves many calls (e.g. every layer of one decode step)."""
+    d = workloads.build(4, 2, 16, ("list", [9000, 70, 0, 2049]), seed=73, causal=True)
+    g = to_dev(d, dev)
+    dec = bd.MlaDecoder(4, 2, 16, g["kv_cache"].shape[0], g["block_table"].shape[1], True, 0, dev)
+    dec.plan(g["cache_seqlens"])
+    outs = []
+    for _ in range(3):
+        out, lse = dec(g["q"], g["kv_cache"], g["block_table"], g["cache_seqlens"], g["softmax_scale"])
+        torch.cuda.synchronize()
+        outs.append((out.clone(), lse.clone()))
+    assert dec.status() == 0
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+    ro, rl = ref(d)
+    helpers.compare(outs[0][0], outs[0][1], ro, rl)
+
+
 def test_single_cta_walks_many_items(dev):
     lens = [130, 1, 64, 900, 65, 3, 2048, 640]
     d = workloads.build(len(lens), 2, 16, ("list", lens), seed=81, causal=True)
