@@ -3,7 +3,8 @@
 
 A step is one pass of the whole hot path over one batch: the split-KV
 schedule, the persistent decode kernel and the LSE combine, all launched
-through the C ABI (libmla_decode.so).  Default workload: batch 16, s_q 1,
+through the C ABI (libmla_decode.so) and captured once as a CUDA graph
+that every timed step replays.  Default workload: batch 16, s_q 1,
 16 heads, KV length 65536 (1.21 GB of latent cache per step, larger than L2,
 so no flush is needed between steps).
 
@@ -317,12 +318,35 @@ def run_ours(args, w):
         bd.mla_decode_get_schedule(dims, sl, sched, stream)
         bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, stream)
 
+    def decode_only():
+        bd.mla_decode_fwd(dims_nc, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, stream)
+
     for _ in range(args.warmup):
         if flush is not None:
             flush.fill_(1)
         step()
     torch.cuda.synchronize()
     assert bd.mla_decode_get_status(sched) == 0, "device status after warm-up"
+
+    # One step (schedule, decode, combine with their programmatic
+    # dependencies) is captured as a CUDA graph and replayed, as a serving loop
+    # would; likewise the decode kernel alone for its roofline timing.
+    g_step = torch.cuda.CUDAGraph()
+    g_dec = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_step, stream=cap):
+            bd.mla_decode_get_schedule(dims, sl, sched, cap)
+            bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, cap)
+        with torch.cuda.graph(g_dec, stream=cap):
+            bd.mla_decode_fwd(dims_nc, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, cap)
+    stream.wait_stream(cap)
+    for _ in range(max(3, args.warmup)):
+        if flush is not None:
+            flush.fill_(1)
+        g_step.replay()
+    torch.cuda.synchronize()
 
     clocks = ClockSampler(dev.index if world == 1 else local).start()
     steps_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -338,7 +362,7 @@ def run_ours(args, w):
         if flush is not None:
             flush.fill_(i & 0xFF)
             steps_ev[i][0].record(stream)
-        step()
+        g_step.replay()
         if flush is not None:
             steps_ev[i][1].record(stream)
     t_end.record(stream)
@@ -352,20 +376,21 @@ def run_ours(args, w):
     else:
         ms_step = t_start.elapsed_time(t_end) / args.steps
 
-    # Decode kernel alone (same plan, combine left out), bracketed by events,
-    # for the kernel's roofline fraction.
+    # Decode kernel alone (same plan, combine left out), for the kernel's
+    # roofline fraction.
     kern = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(i & 0xFF)
         kern[i][0].record(stream)
-        bd.mla_decode_fwd(dims_nc, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, stream)
+        g_dec.replay()
         kern[i][1].record(stream)
     torch.cuda.synchronize()
     kernel_ms = sum(a.elapsed_time(b) for a, b in kern) / args.steps
     status = bd.mla_decode_get_status(sched)
     assert status == 0, "device status %#x" % status
+    del g_step, g_dec
 
     (ms_step, kernel_ms), total_kv = aggregate_over_ranks([ms_step, kernel_ms], byt["kv"], dev)
 

@@ -18,12 +18,13 @@
 //                 (M = 64 tokens, K-major A and B) into TMEM; the two issuers
 //                 take alternate 64-column boxes into separate accumulators,
 //                 which the softmax adds up.
-//   warp 3        one thread issues GEMM2  O^T[512 x N] += V^T[512 x 64] . P^T
-//                 (4 x M = 128 d_v chunks, MN-major A and B); V^T is the same
-//                 shared-memory page read through a second (MN-major) descriptor.
-//                 Separate issuers let GEMM2 of page j start as soon as P^T(j)
-//                 is ready, independently of when page j+1 lands.
-//   warps 4..7    softmax over the KV axis (one TMEM lane = one token), lazy
+//   warp 3 (, 4)  one thread per warp issues GEMM2  O^T[512 x N] += V^T[512 x 64] . P^T
+//                 (4 x M = 128 d_v chunks, MN-major A and B; with two issuers each
+//                 takes two chunks); V^T is the same shared-memory page read
+//                 through a second (MN-major) descriptor.  Separate issuers let
+//                 GEMM2 of page j start as soon as P^T(j) is ready,
+//                 independently of when page j+1 lands.
+//   last 4 warps  softmax over the KV axis (one TMEM lane = one token), lazy
 //                 rescale of O^T in TMEM, P^T to shared memory as bf16, and the
 //                 epilogue (O = O^T / l transposed back, LSE), either final or
 //                 as an fp32 partial of a split request.
@@ -44,12 +45,21 @@ namespace mla {
 
 constexpr uint32_t kFullMask = 0xffffffffu;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-constexpr int kFwdThreads = 256;  // 8 warps: TMA, 2 GEMM1 issuers, GEMM2 issuer, 4 softmax
+// Warps: TMA producer, kG1Issuers GEMM1 issuers, G2Issuers<NG> GEMM2 issuers,
+// then the 4 softmax warps.  The softmax of NG = 32 needs more than the 224
+// registers per thread a ninth warp would leave, so it keeps one GEMM2 issuer.
 // A single thread issues at most one tcgen05.mma every ~45 cycles, while the
 // tensor pipe accepts small (M=64, N<=64) MMAs roughly every 28 cycles from two
 // issuers; GEMM1 is therefore issued by two threads (warps 1 and 2), each into
 // its own accumulator, boxes alternating between them.
 constexpr int kG1Issuers = 2;
+template <int NG>
+struct FwdWarps {
+    static constexpr int kG2Issuers = NG == 16 ? 2 : 1;
+    static constexpr int kFirstG2 = 1 + kG1Issuers;
+    static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
+    static constexpr int kThreads = 32 * (kFirstSoftmax + 4);
+};
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the running max grows by > 2^8
 constexpr float kLn2 = 0.693147180559945309f;
 // GEMM1 (S^T = K Q^T, K = 576) accumulates into one TMEM accumulator per
@@ -90,6 +100,9 @@ enum TraceTag : unsigned {
     kTrSmMaxDone = 9,   // softmax: page column maxima written (before the exchange)
     kTrSmXchg = 10,     // softmax: exchange complete
     kTrSmPStored = 11,  // softmax: P^T stored
+    kTrSmEpiSum = 12,   // softmax: row sums exchanged (epilogue)
+    kTrSmEpiOut = 13,   // softmax: outputs written (epilogue)
+    kTrSmEpiLse = 14,   // softmax: LSE written (epilogue)
 };
 struct Tracer {
     int cta, role;
@@ -152,7 +165,10 @@ struct FwdSmem {
     static constexpr int kKvOff = 0;
     static constexpr int kQOff = kKvOff + kStages * kStageBytes;
     static constexpr int kPOff = kQOff + kQBytes;
-    static constexpr int kRedOff = kPOff + 2 * kPBytes;       // float [2][NG][4] page maxima
+    static constexpr int kOutRows = 16;                       // output rows (query columns) per staging pass
+    static constexpr int kOutOff = kPOff + 2 * kPBytes;       // staging: [16][512] fp32 (or bf16)
+    static constexpr int kOutBytes = kOutRows * kDv * 4;
+    static constexpr int kRedOff = kOutOff + kOutBytes;       // float [2][NG][4] page maxima
     static constexpr int kSumOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]   row sums
     static constexpr int kBarOff = kSumOff + NG * 4 * 4;
     static constexpr int kNumBars = 24;
@@ -174,7 +190,7 @@ struct FwdSmem {
 enum Bar {
     kKvFull0 = 0, kKvFull1, kKvEmpty0, kKvEmpty1, kQFull, kQEmpty,
     kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
-    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kBarCount
+    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kBarCount
 };
 
 // ------------------------------------------------------------------ waits
@@ -500,7 +516,9 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
 // token row.  k-outer order keeps consecutive MMAs on different accumulators.
 template <int NG>
 __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
-                          uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
+                          uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
+    constexpr int kIssuers = FwdWarps<NG>::kG2Issuers;
+    constexpr int kChunksPer = (kDv / 128) / kIssuers;  // d_v chunks of 128 per issuer
     using L = FwdSmem<NG>;
     constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
     constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : kSwizzle64;
@@ -512,7 +530,9 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     Item item;
     uint32_t s_it = 0, item_it = 0;
     bool ok = true, issued = false;
-    MLA_TRACE_DECL(2);
+#ifdef MLA_TRACE
+    Tracer tracer_(issuer == 0 ? 2 : 0, issuer == 0);
+#endif
     const uint64_t a_desc0 = smem_desc(kv_s, L::kBoxBytes, 1024, kSwizzle128);
     const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NG * 2, kPSwizzle);
     while (ok && it.next(p, bginfo, item)) {
@@ -533,7 +553,8 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             for (int k = 0; k < kPage / 16; ++k) {
                 const uint64_t b = b_st + ((k * 16 * NG * 2) >> 4);
 #pragma unroll
-                for (int ch = 0; ch < kDv / 128; ++ch) {
+                for (int cc = 0; cc < kChunksPer; ++cc) {
+                    const int ch = issuer * kChunksPer + cc;
                     const uint64_t a = a_st + (((2 * ch) * L::kBoxBytes + k * 2048) >> 4);
                     umma_f16(tmem + L::kOCol + ch * NG, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
                 }
@@ -561,11 +582,13 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     const int lane = threadIdx.x & 31;
     const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const int gt = threadIdx.x - 128;                     // 0..127 within the softmax group
+    const int gt = threadIdx.x - 32 * FwdWarps<NG>::kFirstSoftmax;  // 0..127 within the softmax group
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
     float* sred = reinterpret_cast<float*>(smem + L::kSumOff);
     uint8_t* pbuf = smem + L::kPOff;
+    float* stage_f32 = reinterpret_cast<float*>(smem + L::kOutOff);
+    __nv_bfloat16* stage_bf16 = reinterpret_cast<__nv_bfloat16*>(smem + L::kOutOff);
     // Token row of this thread in the page (M=64 accumulator: token m sits in
     // TMEM lane 32*(m/16) + m%16) and its column parity.
     const int par = half_parity(lane);
@@ -589,7 +612,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     WorkIter it;
     it.init(meta);
     Item item;
-    uint32_t s_it = 0, item_it = 0;
+    uint32_t s_it = 0, item_it = 0, out_it = 0;
     bool ok = true;
     while (ok && it.next(p, bginfo, item)) {
         int lvis[W];                                      // visible length of each own column
@@ -763,62 +786,103 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         mbar_arrive(bar0 + 8 * kSumFull);
         ok = wait_warp(bar0 + 8 * kSumFull, item_it & 1, ctl);
         if (!ok) break;
-        float lsum[NG], inv[NG];
+        MLA_TRACE_SM(kTrSmEpiSum);
+        // l per column; one thread per column writes its LSE.  The column of
+        // thread gt is picked by a select chain rather than by unrolling the
+        // whole LSE computation per column: this code runs once per item, so
+        // its size (instruction fetch) matters more than its instruction count.
+        float inv[NG], m_gt = -INFINITY, l_gt = 0.f;
 #pragma unroll
         for (int n = 0; n < NG; ++n) {
             const float4 s4 = *reinterpret_cast<const float4*>(sred + n * 4);
-            lsum[n] = (s4.x + s4.y) + (s4.z + s4.w);
-            inv[n] = lsum[n] > 0.f ? 1.f / lsum[n] : 0.f;
+            const float ls = (s4.x + s4.y) + (s4.z + s4.w);
+            inv[n] = ls > 0.f ? rcp_approx(ls) : 0.f;
+            m_gt = gt == n ? m_all[n] : m_gt;
+            l_gt = gt == n ? ls : l_gt;
         }
-#pragma unroll 1
-        for (int ch = 0; ch < kDv / 128; ++ch) {
-            float o[NG];
-            tmem_load_cols<NG>(tmem + lane_base + L::kOCol + ch * NG, o);
-            tmem_ld_wait();
-            const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
-#pragma unroll
-            for (int q = 0; q < NG; ++q) {
-                const int n = pos_to_col(q, NG);
-                const int gc = item.g * NG + n;
-                if (gc < p.N) {
-                    const float v = o[q] * inv[n];
-                    if (item.unsplit) {
-                        const int sq = gc / p.heads;
-                        const int head = gc - sq * p.heads;
-                        p.out[(((size_t)item.b * p.s_q + sq) * p.heads + head) * kDv + d] =
-                            __float2bfloat16_rn(v);
-                    } else if (item.slot >= 0) {
-                        p.opart[((size_t)item.slot * NG + n) * kDv + d] = v;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int n = 0; n < NG; ++n) {
-            const int gc = item.g * NG + n;
-            if (gt == n && gc < p.N) {
-                const float lse2 = lsum[n] > 0.f ? m_all[n] + log2f(lsum[n]) : -INFINITY;
-                const float lse = lse2 * kLn2;
+        {
+            const int gc = item.g * NG + gt;
+            if (gt < NG && gc < p.N) {
+                const float lse = l_gt > 0.f ? (m_gt + log2f(l_gt)) * kLn2 : -INFINITY;
                 if (item.unsplit) {
                     const int sq = gc / p.heads;
                     const int head = gc - sq * p.heads;
                     p.lse[((size_t)item.b * p.heads + head) * p.s_q + sq] = lse;
                 } else if (item.slot >= 0) {
-                    p.lpart[(size_t)item.slot * NG + n] = lse;
+                    p.lpart[(size_t)item.slot * NG + gt] = lse;
                 }
             }
         }
+        MLA_TRACE_SM(kTrSmEpiLse);
+        // O = O^T / l, transposed back through a shared-memory staging tile of
+        // 16 query columns x 512 (bf16 final rows or fp32 partial rows), then
+        // written by one bulk copy: a request's output rows, and a partial
+        // slot, are contiguous in global memory.
+#pragma unroll
+        for (int ps = 0; ps < NG / L::kOutRows; ++ps) {
+            ok = wait_warp(bar0 + 8 * kOutFree, (out_it & 1) ^ 1, ctl);
+            if (!ok) break;
+            const bool f32 = !item.unsplit;
+#pragma unroll 1
+            for (int ch = 0; ch < kDv / 128; ++ch) {
+                // positions 8ps.. hold even columns 16ps + 2i, NG/2 + 8ps.. the odd ones
+                float ev[8], od[8];
+                const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
+                tmem_ld_x8(ta + 8 * ps, ev);
+                tmem_ld_x8(ta + NG / 2 + 8 * ps, od);
+                tmem_ld_wait();
+                const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float ve = ev[i] * inv[16 * ps + 2 * i];
+                    const float vo = od[i] * inv[16 * ps + 2 * i + 1];
+                    if (f32) {
+                        stage_f32[(2 * i) * kDv + d] = ve;
+                        stage_f32[(2 * i + 1) * kDv + d] = vo;
+                    } else {
+                        stage_bf16[(2 * i) * kDv + d] = __float2bfloat16_rn(ve);
+                        stage_bf16[(2 * i + 1) * kDv + d] = __float2bfloat16_rn(vo);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar0 + 8 * kOutStaged);
+            if (gt == 0) {
+                ok = wait_bounded(bar0 + 8 * kOutStaged, out_it & 1, ctl);
+                if (ok) {
+                    const int c0 = item.g * NG + L::kOutRows * ps;  // first query column of the pass
+                    if (f32) {
+                        if (item.slot >= 0)
+                            bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * kDv,
+                                           smem_addr(stage_f32), L::kOutRows * kDv * 4);
+                    } else {
+                        int rows = p.N - c0;
+                        rows = rows < L::kOutRows ? rows : L::kOutRows;
+                        if (rows > 0)
+                            bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * kDv, smem_addr(stage_bf16),
+                                           rows * kDv * 2);
+                    }
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                mbar_arrive(bar0 + 8 * kOutFree);
+            }
+            ++out_it;
+        }
+        if (!ok) break;
+        MLA_TRACE_SM(kTrSmEpiOut);
         if (!item.unsplit && item.slot < 0 && gt == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         MLA_TRACE_SM(kTrSmEpi1);
         tc_fence_before();
         mbar_arrive(bar0 + 8 * kOEmpty);
         ++item_it;
     }
+    if (gt == 0) bulk_wait_all();  // output copies complete before the CTA exits
 }
 
 // ------------------------------------------------------------------ kernels
 template <int NG>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
     mla_decode_fwd_kernel(const __grid_constant__ CUtensorMap kv_map,
                           const __grid_constant__ CUtensorMap q_map, const FwdParams p) {
     using L = FwdSmem<NG>;
@@ -847,9 +911,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < kBarCount; ++i) {
             uint32_t count = 1;
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
-                i == kRedFull0 || i == kRedFull1 || i == kSumFull)
+                i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged)
                 count = 128;
             if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = kG1Issuers;
+            if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
+                count = FwdWarps<NG>::kG2Issuers;
             mbar_init(bar0 + 8 * i, count);
         }
         *abort_flag = 0;
@@ -873,8 +939,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp <= kG1Issuers) {
         if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
-    } else if (warp == kG1Issuers + 1) {
-        if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl);
+    } else if (warp < FwdWarps<NG>::kFirstSoftmax) {
+        if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG>::kFirstG2);
     } else {
         run_softmax<NG>(p, meta, bginfo, smem, tmem, ctl);
     }

@@ -147,7 +147,7 @@ int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const
     if (rc != MLA_OK) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.G);
-    cfg.blockDim = dim3(kFwdThreads);
+    cfg.blockDim = dim3(FwdWarps<NG>::kThreads);
     cfg.dynamicSmemBytes = FwdSmem<NG>::kAlloc;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

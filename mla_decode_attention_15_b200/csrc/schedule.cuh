@@ -25,7 +25,10 @@ constexpr int kPage = 64;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kItemOverhead = 1;   // units charged per (request, head group)
-constexpr int kMinPagesPerCta = 2; // smallest range worth its own CTA
+#ifndef MLA_MIN_PAGES_PER_CTA
+#define MLA_MIN_PAGES_PER_CTA 2
+#endif
+constexpr int kMinPagesPerCta = MLA_MIN_PAGES_PER_CTA;  // smallest range worth its own CTA
 
 // ---- schedule buffer layout (int32 words) ----
 constexpr int kSchedMagic = 0x4D4C4144;  // 'MLAD'
