@@ -952,11 +952,45 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
     }
 }
 
-// LSE-weighted merge of split partials; one CTA per (request-group, column).
-__global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombineParams p) {
+// LSE-weighted merge of split partials; one CTA per (request-group, column),
+// four output columns d per thread.  After the decode grid completes, the
+// merge is one round of loads: the k partial LSEs are read one per thread and
+// reduced across the block while the first kCombinePre partial rows are
+// already in flight; further rows are read kCombineUnroll at a time.
+constexpr int kCombineThreads = kDv / 4;
+constexpr int kCombinePre = 8;
+constexpr int kCombineUnroll = 8;
+
+template <bool kMax>
+__device__ __forceinline__ float combine_block_reduce(float v, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float y = __shfl_xor_sync(kFullMask, v, o);
+        v = kMax ? fmaxf(v, y) : v + y;
+    }
+    __syncthreads();  // red[] of an earlier reduction has been read
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    v = red[0];
+#pragma unroll
+    for (int w = 1; w < kCombineThreads / 32; ++w) v = kMax ? fmaxf(v, red[w]) : v + red[w];
+    return v;
+}
+
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
+}
+
+__global__ void __launch_bounds__(kCombineThreads) mla_decode_combine_kernel(const CombineParams p) {
+    __shared__ float red[kCombineThreads / 32];
+    __shared__ float wts[kCombineThreads];
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
-    griddep_wait();  // the decode grid's partials are complete and visible
+    // The plan may be read before the wait: the decode grid let this grid
+    // start only after its own wait on the grid that wrote the plan.
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
         __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != p.NG) {
@@ -970,7 +1004,7 @@ __global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombinePa
     const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
     const int base = __ldg(info + 0);
     const int k = __ldg(info + 1);
-    if (k == 1) return;
+    if (k == 1) return;  // unsplit: the decode kernel wrote the final row
     if (k > 1 && (base < 0 || base + k > p.slots_cap)) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
@@ -978,24 +1012,52 @@ __global__ void __launch_bounds__(128) mla_decode_combine_kernel(const CombinePa
     const int s = gc / p.heads;
     const int head = gc - s * p.heads;
     const int d0 = threadIdx.x * 4;
+    const float* lp = p.lpart + (size_t)base * p.NG + n;
+    const float* op = p.opart + ((size_t)base * p.NG + n) * kDv + d0;
+    const size_t ostride = (size_t)p.NG * kDv;
+    griddep_wait();  // the decode grid's partials are complete and visible
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lstar = -INFINITY;
     if (k > 1) {
-        const float* lp = p.lpart + (size_t)base * p.NG + n;
-        float mx = -INFINITY;
-        for (int i = 0; i < k; ++i) mx = fmaxf(mx, __ldg(lp + (size_t)i * p.NG));
-        if (mx != -INFINITY) {
+        float4 pre[kCombinePre];
+#pragma unroll
+        for (int i = 0; i < kCombinePre; ++i)
+            if (i < k) pre[i] = __ldg(reinterpret_cast<const float4*>(op + (size_t)i * ostride));
+        float own = threadIdx.x < k ? __ldg(lp + (size_t)threadIdx.x * p.NG) : -INFINITY;
+        float mx = own;
+        for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads)
+            mx = fmaxf(mx, __ldg(lp + (size_t)i * p.NG));
+        mx = combine_block_reduce<true>(mx, red);
+        if (mx != -INFINITY) {  // uniform across the block
             float sum = 0.f;
-            for (int i = 0; i < k; ++i) sum += expf(__ldg(lp + (size_t)i * p.NG) - mx);
+            for (int i = threadIdx.x; i < k; i += kCombineThreads)
+                sum += expf((i == threadIdx.x ? own : __ldg(lp + (size_t)i * p.NG)) - mx);
+            sum = combine_block_reduce<false>(sum, red);
             lstar = mx + logf(sum);
-            const float* op = p.opart + ((size_t)base * p.NG + n) * kDv + d0;
-            for (int i = 0; i < k; ++i) {
-                const float w = expf(__ldg(lp + (size_t)i * p.NG) - lstar);
-                const float4 v = __ldg(reinterpret_cast<const float4*>(op + (size_t)i * p.NG * kDv));
-                acc.x += w * v.x;
-                acc.y += w * v.y;
-                acc.z += w * v.z;
-                acc.w += w * v.w;
+            for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
+                const int cn = k - c0 < kCombineThreads ? k - c0 : kCombineThreads;
+                __syncthreads();  // the previous chunk's weights are consumed
+                if (threadIdx.x < cn)
+                    wts[threadIdx.x] =
+                        expf((c0 == 0 ? own : __ldg(lp + (size_t)(c0 + threadIdx.x) * p.NG)) - lstar);
+                __syncthreads();
+                int i = 0;
+                if (c0 == 0) {
+#pragma unroll
+                    for (int j = 0; j < kCombinePre; ++j)
+                        if (j < cn) fma4(acc, wts[j], pre[j]);
+                    i = cn < kCombinePre ? cn : kCombinePre;
+                }
+                for (; i + kCombineUnroll <= cn; i += kCombineUnroll) {
+                    float4 v[kCombineUnroll];
+#pragma unroll
+                    for (int j = 0; j < kCombineUnroll; ++j)
+                        v[j] = __ldg(reinterpret_cast<const float4*>(op + (size_t)(c0 + i + j) * ostride));
+#pragma unroll
+                    for (int j = 0; j < kCombineUnroll; ++j) fma4(acc, wts[i + j], v[j]);
+                }
+                for (; i < cn; ++i)
+                    fma4(acc, wts[i], __ldg(reinterpret_cast<const float4*>(op + (size_t)(c0 + i) * ostride)));
             }
         }
     }

@@ -181,7 +181,7 @@ int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedul
     c.slots_cap = (int)pl.slots;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.BG, pl.gr.NG);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(kCombineThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
