@@ -67,6 +67,8 @@ extern "C" {
 #define MLA_STATUS_TIMEOUT 0x2         /* a pipeline wait exceeded its limit; that CTA stopped early */
 #define MLA_STATUS_BAD_SEQLEN 0x4      /* cache_seqlens[b] outside [0, 64*max_blocks_per_seq]; clamped */
 #define MLA_STATUS_BAD_SCHEDULE 0x8    /* schedule header did not match the launch; nothing written */
+#define MLA_STATUS_SMEM_ALIGN 0x10     /* dynamic shared memory base not 1 KB aligned (64-column groups,
+                                          which have no room to realign); nothing written */
 
 /* dims.flags */
 #define MLA_FLAG_NO_COMBINE 0x1 /* mla_decode_fwd does not enqueue the combine; call mla_decode_combine */

@@ -27,6 +27,7 @@ MLA_STATUS_BAD_BLOCK_TABLE = 0x1
 MLA_STATUS_TIMEOUT = 0x2
 MLA_STATUS_BAD_SEQLEN = 0x4
 MLA_STATUS_BAD_SCHEDULE = 0x8
+MLA_STATUS_SMEM_ALIGN = 0x10
 
 MLA_FLAG_NO_COMBINE = 0x1
 

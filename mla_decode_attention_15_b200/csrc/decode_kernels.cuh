@@ -55,12 +55,27 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 // ~15% sooner than from one thread in this kernel (bs16 x 64K: 214.5 vs
 // 247.3 us per launch, B200); per-box "landed" barriers did not help.
 constexpr int kG1Issuers = 2;
+// 64-column groups run 8 softmax warps: two column groups of 32 columns,
+// each the 4 warps that reach the four TMEM lane quadrants.  Their 384
+// threads leave 168 registers per thread at launch; warpgroup 0 (producer and
+// issuers) gives registers back with setmaxnreg so that the softmax
+// warpgroups can hold the per-column state of 32 columns.
 template <int NG>
 struct FwdWarps {
     static constexpr int kG2Issuers = NG == 16 ? 2 : 1;
     static constexpr int kFirstG2 = 1 + kG1Issuers;
     static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
-    static constexpr int kThreads = 32 * (kFirstSoftmax + 4);
+    static constexpr int kColGroups = NG == 64 ? 2 : 1;   // softmax column groups
+    static constexpr int kGroupCols = NG / kColGroups;     // query columns per group
+    static constexpr int kSoftmaxThreads = 128 * kColGroups;
+    static constexpr int kThreads = 32 * kFirstSoftmax + kSoftmaxThreads;
+    static constexpr bool kSplitRegs = NG == 64;
+    static constexpr int kRegsLaunch = 168;                 // 65536 / 384, rounded down to 8
+    static constexpr int kRegsIssue = 56;                   // warpgroup 0 after setmaxnreg.dec
+    static constexpr int kRegsSoftmax = 224;                // softmax warpgroups after setmaxnreg.inc
+    static_assert(!kSplitRegs || (kFirstSoftmax == 4 && kThreads == 384), "warpgroup 0 = producer + issuers");
+    static_assert(!kSplitRegs || kRegsIssue * 128 + kRegsSoftmax * kSoftmaxThreads <= kRegsLaunch * kThreads,
+                  "register split exceeds the launch allocation");
 };
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the running max grows by > 2^8
 constexpr float kLn2 = 0.693147180559945309f;
@@ -166,19 +181,26 @@ struct FwdSmem {
     static constexpr int kQBoxBytes = NG * 128;               // NG rows x 64 cols
     static constexpr int kQBytes = kBoxes * kQBoxBytes;
     static constexpr int kPBytes = kPage * NG * 2;            // P^T of one page, bf16
+    // 64-column groups: Q^T takes 72 KB, so P^T is single-buffered and the
+    // epilogue stores straight from registers (no staging tile).
+    static constexpr int kPBuffers = NG == 64 ? 1 : 2;
     static constexpr int kKvOff = 0;
     static constexpr int kQOff = kKvOff + kStages * kStageBytes;
     static constexpr int kPOff = kQOff + kQBytes;
-    static constexpr int kOutRows = 16;                       // output rows (query columns) per staging pass
-    static constexpr int kOutOff = kPOff + 2 * kPBytes;       // staging: [16][512] fp32 (or bf16)
+    static constexpr int kOutRows = NG == 64 ? 0 : 16;        // output rows (query columns) per staging pass
+    static constexpr int kOutOff = kPOff + kPBuffers * kPBytes;  // staging: [16][512] fp32 (or bf16)
     static constexpr int kOutBytes = kOutRows * kDv * 4;
-    static constexpr int kRedOff = kOutOff + kOutBytes;       // float [2][NG][4] page maxima
-    static constexpr int kSumOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]   row sums
-    static constexpr int kBarOff = kSumOff + NG * 4 * 4;
+    // float [2][NG][4]: page maxima of the 4 lane quadrants, double-buffered
+    // by page; the epilogue's row sums use the buffer of the item's last page.
+    static constexpr int kRedOff = kOutOff + kOutBytes;
+    static constexpr int kBarOff = kRedOff + 2 * NG * 4 * 4;
     static constexpr int kNumBars = 24;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMiscOff + 16;
-    static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KB
+    // Slack to align the base to 1 KB where it fits; without it the kernel
+    // checks that the dynamic shared memory base is 1 KB aligned.
+    static constexpr int kAlignSlack = kBytes + 1024 <= 227 * 1024 ? 1024 : 0;
+    static constexpr int kAlloc = kBytes + kAlignSlack;
     // TMEM columns: S^T buffer i, chain c at kSCol + (i*kSChains + c)*NG;
     // O^T d_v chunk c at kOCol + c*NG.
     static constexpr int kSCol = 0;
@@ -196,6 +218,7 @@ enum Bar {
     kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
     kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kBarCount
 };
+static_assert(kBarCount <= FwdSmem<16>::kNumBars, "barrier slots");
 
 // ------------------------------------------------------------------ waits
 struct Ctl {
@@ -526,7 +549,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     constexpr int kChunksPer = (kDv / 128) / kIssuers;  // d_v chunks of 128 per issuer
     using L = FwdSmem<NG>;
     constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
-    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : kSwizzle64;
+    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : NG == 32 ? kSwizzle64 : kSwizzle128;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t p_s = smem_addr(smem + L::kPOff);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
@@ -543,8 +566,9 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     while (ok && it.next(p, bginfo, item)) {
         for (int j = item.p0; j < item.p1; ++j) {
             const int st = s_it & 1;
+            const int pb = s_it % L::kPBuffers;
             const bool first = (j == item.p0);
-            ok = wait_bounded(bar0 + 8 * (kPFull0 + st), (s_it >> 1) & 1, ctl);
+            ok = wait_bounded(bar0 + 8 * (kPFull0 + pb), (s_it / L::kPBuffers) & 1, ctl);
             if (!ok) break;
             if (first) {
                 ok = wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl);
@@ -553,7 +577,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             MLA_TRACE_EV(kTrMmaPFull);
             tc_fence_after();
             const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
-            const uint64_t b_st = b_desc0 + ((st * L::kPBytes) >> 4);
+            const uint64_t b_st = b_desc0 + ((pb * L::kPBytes) >> 4);
 #pragma unroll
             for (int k = 0; k < kPage / 16; ++k) {
                 const uint64_t b = b_st + ((k * 16 * NG * 2) >> 4);
@@ -566,7 +590,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             }
             issued = true;
             umma_commit(bar0 + 8 * (kKvEmpty0 + st));
-            umma_commit(bar0 + 8 * (kPEmpty0 + st));
+            umma_commit(bar0 + 8 * (kPEmpty0 + pb));
             MLA_TRACE_EV(kTrMmaG2Issued);
             ++s_it;
         }
@@ -583,15 +607,20 @@ template <int NG>
 __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                             uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
     using L = FwdSmem<NG>;
-    constexpr int W = NG / 2;                             // own columns per thread
+    using Wp = FwdWarps<NG>;
+    constexpr int NGW = Wp::kGroupCols;                   // query columns of this warp's group
+    constexpr int W = NGW / 2;                            // own columns per thread
+    constexpr int kPB = L::kPBuffers;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
+    const int cg = (warp - Wp::kFirstSoftmax) >> 2;       // column group: columns [cg*NGW, cg*NGW + NGW)
+    const int c0g = cg * NGW;
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const int gt = threadIdx.x - 32 * FwdWarps<NG>::kFirstSoftmax;  // 0..127 within the softmax group
+    const int gt = threadIdx.x - 32 * Wp::kFirstSoftmax;  // 0 .. kSoftmaxThreads-1
+    const int gtg = gt & 127;                             // 0..127 within the column group
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
-    float* sred = reinterpret_cast<float*>(smem + L::kSumOff);
     uint8_t* pbuf = smem + L::kPOff;
     float* stage_f32 = reinterpret_cast<float*>(smem + L::kOutOff);
     __nv_bfloat16* stage_bf16 = reinterpret_cast<__nv_bfloat16*>(smem + L::kOutOff);
@@ -599,12 +628,14 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     // TMEM lane 32*(m/16) + m%16) and its column parity.
     const int par = half_parity(lane);
     const int row = 16 * wq + half_token(lane);
-    const int red_i = half_reduced_index<NG>(lane);
-    const int red_col = par + 2 * red_i;
-    const bool red_w = half_reduced_writer<NG>(lane);
-    // P^T row: W bf16 at positions par*W .. par*W+W-1, in 16-byte chunks.
+    const int red_i = half_reduced_index<NGW>(lane);
+    const int red_col = c0g + par + 2 * red_i;            // column whose reduction this thread holds
+    const bool red_w = half_reduced_writer<NGW>(lane);
+    // P^T row: NG bf16 positions; the group owns positions c0g .. c0g+NGW-1,
+    // parity-major inside (own columns of parity par at c0g + par*W ..).
     constexpr int kChunks = NG * 2 / 16;                  // 16-byte chunks per P^T row
-    constexpr int kMyChunks = kChunks / 2;
+    constexpr int kMyChunks = NGW / 16;                   // chunks of one thread
+    const int chunk0 = cg * (NGW / 8) + par * kMyChunks;
     const int swz = ((row * NG * 2) >> 7) & (kChunks - 1);
 #ifdef MLA_TRACE
     Tracer tracer_(3);
@@ -624,7 +655,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         int lvis[W];                                      // visible length of each own column
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-            const int gc = item.g * NG + par + 2 * i;
+            const int gc = item.g * NG + c0g + par + 2 * i;
             int v = 0;
             if (gc < p.N) {
                 const int sq = gc / p.heads;
@@ -632,10 +663,10 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             }
             lvis[i] = v;
         }
-        float m_all[NG];                                  // running max (log2 units), every column
+        float m_all[NGW];                                 // running max (log2 units), every group column
         float l_own[W];                                   // running row sum, own columns, own token
 #pragma unroll
-        for (int n = 0; n < NG; ++n) m_all[n] = -INFINITY;
+        for (int n = 0; n < NGW; ++n) m_all[n] = -INFINITY;
 #pragma unroll
         for (int i = 0; i < W; ++i) l_own[i] = 0.f;
 
@@ -647,12 +678,12 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             tc_fence_after();
             float x[W];
             {
-                const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG;
-                tmem_load_half<NG>(sbase, x);
+                const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG + c0g;
+                tmem_load_half<NGW>(sbase, x);
 #pragma unroll
                 for (int c = 1; c < kSChains; ++c) {
                     float y[W];
-                    tmem_load_half<NG>(sbase + c * NG, y);
+                    tmem_load_half<NGW>(sbase + c * NG, y);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < W; ++i) x[i] += y[i];
@@ -667,7 +698,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             for (int i = 0; i < W; ++i) x[i] = (t < lvis[i]) ? x[i] * p.scale_log2 : -INFINITY;
 
             // Page maxima of the own columns over the 16 tokens of this warp,
-            // then the four warps meet through shared memory.
+            // then the four warps of the group meet through shared memory.
             float* rb = red + (s_it & 1) * NG * 4;
             {
                 float xr[W];
@@ -687,7 +718,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             float e[W];
 #pragma unroll
             for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
-            const int pb = s_it & 1;
+            const int pb = s_it % kPB;
             uint8_t* rowp = pbuf + pb * L::kPBytes + row * (NG * 2);
             auto store_p = [&](const float (&ev)[W]) {
                 uint32_t packed[W / 2];
@@ -698,12 +729,12 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 }
 #pragma unroll
                 for (int c = 0; c < kMyChunks; ++c) {
-                    const int chunk = par * kMyChunks + c;
+                    const int chunk = chunk0 + c;
                     *reinterpret_cast<uint4*>(rowp + ((chunk ^ swz) * 16)) =
                         make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
                 }
             };
-            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
+            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it / kPB) & 1) ^ 1, ctl);
             if (!ok) break;
             store_p(e);
             fence_proxy_async_smem();
@@ -715,22 +746,23 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             bool grow = false;
 #pragma unroll
             for (int i = 0; i < W; ++i) {
-                const float4 r4 = *reinterpret_cast<const float4*>(rb + (par + 2 * i) * 4);
+                const float4 r4 = *reinterpret_cast<const float4*>(rb + (c0g + par + 2 * i) * 4);
                 const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
                 grow |= pmax > m_own[i] + kRescaleLog2;
             }
-            // The warp's threads cover every column and every warp reads the
-            // same maxima, so this decision is uniform across the CTA.
+            // The warp's threads cover every column of the group and the
+            // group's four warps read the same maxima, so this decision is
+            // uniform across the group.
             if (!__any_sync(kFullMask, grow)) {
 #pragma unroll
                 for (int i = 0; i < W; ++i) l_own[i] += e[i];
             } else {
                 // Slow path (first page of an item, or a jump of the max):
                 // move the reference max of the grown columns, rescale.
-                float alpha[NG];
+                float alpha[NGW];
 #pragma unroll
-                for (int n = 0; n < NG; ++n) {
-                    const float4 r4 = *reinterpret_cast<const float4*>(rb + n * 4);
+                for (int n = 0; n < NGW; ++n) {
+                    const float4 r4 = *reinterpret_cast<const float4*>(rb + (c0g + n) * 4);
                     const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
                     const float mnew = fmaxf(m_all[n], pmax);
                     if (mnew > m_all[n] + kRescaleLog2) {
@@ -751,20 +783,24 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 fence_proxy_async_smem();
                 if (j > item.p0) {
                     // O^T already holds earlier pages: wait for the previous
-                    // GEMM2, then scale each column (position) in place.
+                    // GEMM2, then scale each of the group's columns (positions)
+                    // in place.
                     const uint32_t prev = s_it - 1;
-                    ok = wait_warp(bar0 + 8 * (kPEmpty0 + (prev & 1)), (prev >> 1) & 1, ctl);
+                    ok = wait_warp(bar0 + 8 * (kPEmpty0 + prev % kPB), (prev / kPB) & 1, ctl);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
                     for (int ch = 0; ch < kDv / 128; ++ch) {
-                        float o[NG];
-                        const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
-                        tmem_load_cols<NG>(ta, o);
-                        tmem_ld_wait();
 #pragma unroll
-                        for (int q = 0; q < NG; ++q) o[q] *= alpha[pos_to_col(q, NG)];
-                        tmem_store_cols<NG>(ta, o);
+                        for (int h = 0; h < NGW; h += 16) {  // 16 positions at a time
+                            float o[16];
+                            const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG + c0g + h;
+                            tmem_ld_x16(ta, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) o[q] *= alpha[pos_to_col(h + q, NGW)];
+                            tmem_st_x16(ta, o);
+                        }
                     }
                     tmem_st_wait();
                 }
@@ -778,10 +814,15 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 
         // ---- epilogue: wait for the last GEMM2, reduce l over the tokens ----
         const uint32_t last = s_it - 1;
-        ok = wait_warp(bar0 + 8 * (kPEmpty0 + (last & 1)), (last >> 1) & 1, ctl);
+        ok = wait_warp(bar0 + 8 * (kPEmpty0 + last % kPB), (last / kPB) & 1, ctl);
         if (!ok) break;
         MLA_TRACE_SM(kTrSmEpi0);
         tc_fence_after();
+        // Row sums go through the page-maxima buffer of the last page: every
+        // thread has read it (the last GEMM2 waited for all of them), and the
+        // next write to it is two pages on, after all threads have left this
+        // epilogue.
+        float* sred = red + (last & 1) * NG * 4;
         {
             float lr[W];
 #pragma unroll
@@ -793,89 +834,119 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         ok = wait_warp(bar0 + 8 * kSumFull, item_it & 1, ctl);
         if (!ok) break;
         MLA_TRACE_SM(kTrSmEpiSum);
-        // l per column; one thread per column writes its LSE.  The column of
-        // thread gt is picked by a select chain rather than by unrolling the
-        // whole LSE computation per column: this code runs once per item, so
-        // its size (instruction fetch) matters more than its instruction count.
-        float inv[NG], m_gt = -INFINITY, l_gt = 0.f;
+        // l per group column; one thread per column writes its LSE.  The
+        // column of thread gtg is picked by a select chain rather than by
+        // unrolling the whole LSE computation per column: this code runs once
+        // per item, so its size (instruction fetch) matters more than its
+        // instruction count.
+        float inv[NGW], m_gt = -INFINITY, l_gt = 0.f;
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sred + n * 4);
+        for (int n = 0; n < NGW; ++n) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sred + (c0g + n) * 4);
             const float ls = (s4.x + s4.y) + (s4.z + s4.w);
             inv[n] = ls > 0.f ? rcp_approx(ls) : 0.f;
-            m_gt = gt == n ? m_all[n] : m_gt;
-            l_gt = gt == n ? ls : l_gt;
+            m_gt = gtg == n ? m_all[n] : m_gt;
+            l_gt = gtg == n ? ls : l_gt;
         }
         {
-            const int gc = item.g * NG + gt;
-            if (gt < NG && gc < p.N) {
+            const int gc = item.g * NG + c0g + gtg;
+            if (gtg < NGW && gc < p.N) {
                 const float lse = l_gt > 0.f ? (m_gt + log2f(l_gt)) * kLn2 : -INFINITY;
                 if (item.unsplit) {
                     const int sq = gc / p.heads;
                     const int head = gc - sq * p.heads;
                     p.lse[((size_t)item.b * p.heads + head) * p.s_q + sq] = lse;
                 } else if (item.slot >= 0) {
-                    p.lpart[(size_t)item.slot * NG + gt] = lse;
+                    p.lpart[(size_t)item.slot * NG + c0g + gtg] = lse;
                 }
             }
         }
         MLA_TRACE_SM(kTrSmEpiLse);
-        // O = O^T / l, transposed back through a shared-memory staging tile of
-        // 16 query columns x 512 (bf16 final rows or fp32 partial rows), then
-        // written by one bulk copy: a request's output rows, and a partial
-        // slot, are contiguous in global memory.
+        if constexpr (L::kOutRows > 0) {
+            // O = O^T / l, transposed back through a shared-memory staging tile of
+            // 16 query columns x 512 (bf16 final rows or fp32 partial rows), then
+            // written by one bulk copy: a request's output rows, and a partial
+            // slot, are contiguous in global memory.
 #pragma unroll
-        for (int ps = 0; ps < NG / L::kOutRows; ++ps) {
-            ok = wait_warp(bar0 + 8 * kOutFree, (out_it & 1) ^ 1, ctl);
+            for (int ps = 0; ps < NG / L::kOutRows; ++ps) {
+                ok = wait_warp(bar0 + 8 * kOutFree, (out_it & 1) ^ 1, ctl);
+                if (!ok) break;
+                const bool f32 = !item.unsplit;
+#pragma unroll 1
+                for (int ch = 0; ch < kDv / 128; ++ch) {
+                    // positions 8ps.. hold even columns 16ps + 2i, NG/2 + 8ps.. the odd ones
+                    float ev[8], od[8];
+                    const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
+                    tmem_ld_x8(ta + 8 * ps, ev);
+                    tmem_ld_x8(ta + NG / 2 + 8 * ps, od);
+                    tmem_ld_wait();
+                    const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float ve = ev[i] * inv[16 * ps + 2 * i];
+                        const float vo = od[i] * inv[16 * ps + 2 * i + 1];
+                        if (f32) {
+                            stage_f32[(2 * i) * kDv + d] = ve;
+                            stage_f32[(2 * i + 1) * kDv + d] = vo;
+                        } else {
+                            stage_bf16[(2 * i) * kDv + d] = __float2bfloat16_rn(ve);
+                            stage_bf16[(2 * i + 1) * kDv + d] = __float2bfloat16_rn(vo);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar0 + 8 * kOutStaged);
+                if (gt == 0) {
+                    ok = wait_bounded(bar0 + 8 * kOutStaged, out_it & 1, ctl);
+                    if (ok) {
+                        const int c0 = item.g * NG + L::kOutRows * ps;  // first query column of the pass
+                        if (f32) {
+                            if (item.slot >= 0)
+                                bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * kDv,
+                                               smem_addr(stage_f32), L::kOutRows * kDv * 4);
+                        } else {
+                            int rows = p.N - c0;
+                            rows = rows < L::kOutRows ? rows : L::kOutRows;
+                            if (rows > 0)
+                                bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * kDv, smem_addr(stage_bf16),
+                                               rows * kDv * 2);
+                        }
+                        bulk_commit();
+                        bulk_wait_read_all();
+                    }
+                    mbar_arrive(bar0 + 8 * kOutFree);
+                }
+                ++out_it;
+            }
             if (!ok) break;
+        } else {
+            // No staging room: O = O^T / l straight from registers.  For one
+            // query column the 32 lanes of a warp hold 32 consecutive d, so
+            // each store instruction writes 64 (bf16) or 128 (fp32) contiguous
+            // bytes.
             const bool f32 = !item.unsplit;
 #pragma unroll 1
             for (int ch = 0; ch < kDv / 128; ++ch) {
-                // positions 8ps.. hold even columns 16ps + 2i, NG/2 + 8ps.. the odd ones
-                float ev[8], od[8];
-                const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
-                tmem_ld_x8(ta + 8 * ps, ev);
-                tmem_ld_x8(ta + NG / 2 + 8 * ps, od);
-                tmem_ld_wait();
-                const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float ve = ev[i] * inv[16 * ps + 2 * i];
-                    const float vo = od[i] * inv[16 * ps + 2 * i + 1];
+              for (int h = 0; h < NGW; h += 16) {  // 16 positions at a time
+                float o[16];
+                tmem_ld_x16(tmem + lane_base + L::kOCol + ch * NG + c0g + h, o);
+                tmem_ld_wait();
+                const int d = ch * 128 + 32 * wq + lane;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int n = pos_to_col(h + q, NGW);          // group column of position h + q
+                    const float v = o[q] * inv[n];
                     if (f32) {
-                        stage_f32[(2 * i) * kDv + d] = ve;
-                        stage_f32[(2 * i + 1) * kDv + d] = vo;
+                        if (item.slot >= 0) p.opart[((size_t)item.slot * NG + c0g + n) * kDv + d] = v;
                     } else {
-                        stage_bf16[(2 * i) * kDv + d] = __float2bfloat16_rn(ve);
-                        stage_bf16[(2 * i + 1) * kDv + d] = __float2bfloat16_rn(vo);
+                        const int gc = item.g * NG + c0g + n;
+                        if (gc < p.N) p.out[((size_t)item.b * p.N + gc) * kDv + d] = __float2bfloat16_rn(v);
                     }
                 }
+              }
             }
-            fence_proxy_async_smem();
-            mbar_arrive(bar0 + 8 * kOutStaged);
-            if (gt == 0) {
-                ok = wait_bounded(bar0 + 8 * kOutStaged, out_it & 1, ctl);
-                if (ok) {
-                    const int c0 = item.g * NG + L::kOutRows * ps;  // first query column of the pass
-                    if (f32) {
-                        if (item.slot >= 0)
-                            bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * kDv,
-                                           smem_addr(stage_f32), L::kOutRows * kDv * 4);
-                    } else {
-                        int rows = p.N - c0;
-                        rows = rows < L::kOutRows ? rows : L::kOutRows;
-                        if (rows > 0)
-                            bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * kDv, smem_addr(stage_bf16),
-                                           rows * kDv * 2);
-                    }
-                    bulk_commit();
-                    bulk_wait_read_all();
-                }
-                mbar_arrive(bar0 + 8 * kOutFree);
-            }
-            ++out_it;
         }
-        if (!ok) break;
         MLA_TRACE_SM(kTrSmEpiOut);
         if (!item.unsplit && item.slot < 0 && gt == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         MLA_TRACE_SM(kTrSmEpi1);
@@ -883,7 +954,8 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         mbar_arrive(bar0 + 8 * kOEmpty);
         ++item_it;
     }
-    if (gt == 0) bulk_wait_all();  // output copies complete before the CTA exits
+    if constexpr (L::kOutRows > 0)
+        if (gt == 0) bulk_wait_all();  // output copies complete before the CTA exits
 }
 
 // ------------------------------------------------------------------ kernels
@@ -907,6 +979,12 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
+    if constexpr (L::kAlignSlack == 0) {
+        if (smem != smem_raw) {  // no room was reserved to realign the base
+            if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_SMEM_ALIGN);
+            return;
+        }
+    }
     const int32_t* meta = hdr + kHdrWords + (size_t)blockIdx.x * kMetaWords;
     const int32_t* bginfo = hdr + bg_offset_words(p.G);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
@@ -918,7 +996,7 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
             uint32_t count = 1;
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
                 i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged)
-                count = 128;
+                count = FwdWarps<NG>::kSoftmaxThreads;
             if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = kG1Issuers;
             if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
                 count = FwdWarps<NG>::kG2Issuers;
@@ -937,17 +1015,21 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const Ctl ctl{abort_flag, p.status};
 
-    if (warp == 0) {
-        if (lane == 0) {
-            prefetch_tensormap(&kv_map);
-            prefetch_tensormap(&q_map);
-            run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
+    if (warp < FwdWarps<NG>::kFirstSoftmax) {
+        if constexpr (FwdWarps<NG>::kSplitRegs) setmaxnreg_dec<FwdWarps<NG>::kRegsIssue>();
+        if (warp == 0) {
+            if (lane == 0) {
+                prefetch_tensormap(&kv_map);
+                prefetch_tensormap(&q_map);
+                run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
+            }
+        } else if (warp <= kG1Issuers) {
+            if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
+        } else {
+            if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG>::kFirstG2);
         }
-    } else if (warp <= kG1Issuers) {
-        if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
-    } else if (warp < FwdWarps<NG>::kFirstSoftmax) {
-        if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG>::kFirstG2);
     } else {
+        if constexpr (FwdWarps<NG>::kSplitRegs) setmaxnreg_inc<FwdWarps<NG>::kRegsSoftmax>();
         run_softmax<NG>(p, meta, bginfo, smem, tmem, ctl);
     }
     tc_fence_before();

@@ -135,6 +135,16 @@ int ensure_smem_attr() {
         if (cudaFuncSetAttribute(mla_decode_fwd_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  FwdSmem<NG>::kAlloc) != cudaSuccess)
             return MLA_ERR_CUDA;
+        if constexpr (FwdWarps<NG>::kSplitRegs) {
+            // setmaxnreg.inc waits until the registers it asks for are free in
+            // the CTA, so the split must fit the launch allocation exactly as
+            // compiled; refuse to launch otherwise.
+            using Wp = FwdWarps<NG>;
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, mla_decode_fwd_kernel<NG>) != cudaSuccess) return MLA_ERR_CUDA;
+            if ((long)fa.numRegs * Wp::kThreads < (long)Wp::kRegsIssue * 128 + (long)Wp::kRegsSoftmax * Wp::kSoftmaxThreads)
+                return MLA_ERR_UNSUPPORTED;
+        }
         done[dev] = true;
     }
     return MLA_OK;
@@ -352,7 +362,9 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = pl.gr.NG == 16 ? launch_fwd<16>(pl, p, kvm, qm, st) : launch_fwd<32>(pl, p, kvm, qm, st);
+    rc = pl.gr.NG == 16   ? launch_fwd<16>(pl, p, kvm, qm, st)
+         : pl.gr.NG == 32 ? launch_fwd<32>(pl, p, kvm, qm, st)
+                          : launch_fwd<64>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
     return launch_combine(dims, pl, schedule, workspace, out, lse, st);

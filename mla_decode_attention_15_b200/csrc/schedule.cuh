@@ -77,8 +77,8 @@ __host__ __device__ inline Grouping make_grouping(int heads, int s_q) {
         gr.NG = 32;
         gr.Hg = 1;
     } else {
-        gr.NG = 32;
-        gr.Hg = (gr.N + 31) / 32;
+        gr.NG = 64;
+        gr.Hg = (gr.N + 63) / 64;
     }
     return gr;
 }

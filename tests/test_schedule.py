@@ -24,7 +24,7 @@ def host_plan(seqlens, s_q, heads, G, max_blocks=None):
     n = bd.mla_decode_schedule_bytes(d)
     buf = torch.zeros(n, dtype=torch.uint8)
     bd.mla_decode_get_schedule_host(d, seqlens, buf)
-    Hg = 1 if heads * s_q <= 32 else (heads * s_q + 31) // 32
+    Hg = 1 if heads * s_q <= 64 else (heads * s_q + 63) // 64
     BG = B * Hg
     hdr, meta, bginfo, prefix = helpers.read_plan(buf.numpy(), G, BG)
     return dict(hdr=hdr, meta=meta, bginfo=bginfo, prefix=prefix, Hg=Hg, BG=BG, G=G,
