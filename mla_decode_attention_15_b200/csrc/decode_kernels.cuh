@@ -181,14 +181,18 @@ struct FwdSmem {
     static constexpr int kQBoxBytes = NG * 128;               // NG rows x 64 cols
     static constexpr int kQBytes = kBoxes * kQBoxBytes;
     static constexpr int kPBytes = kPage * NG * 2;            // P^T of one page, bf16
-    // 64-column groups: Q^T takes 72 KB, so P^T is single-buffered and the
-    // epilogue stores straight from registers (no staging tile).
-    static constexpr int kPBuffers = NG == 64 ? 1 : 2;
+    // P^T of a page is written over the page's own RoPE box (box 8): only
+    // GEMM1 reads that box, S^T is complete before the softmax writes P^T, and
+    // the stage is refilled only after the page's GEMM2 has read P^T.  So P^T
+    // is double-buffered with the stages at no cost in shared memory.
+    static constexpr int kPInStage = 8 * kBoxBytes;
+    static_assert(kPBytes <= kBoxBytes, "P^T fits the RoPE box");
     static constexpr int kKvOff = 0;
     static constexpr int kQOff = kKvOff + kStages * kStageBytes;
-    static constexpr int kPOff = kQOff + kQBytes;
+    // 64-column groups: Q^T takes 72 KB, so the epilogue stores straight from
+    // registers (no staging tile).
     static constexpr int kOutRows = NG == 64 ? 0 : 16;        // output rows (query columns) per staging pass
-    static constexpr int kOutOff = kPOff + kPBuffers * kPBytes;  // staging: [16][512] fp32 (or bf16)
+    static constexpr int kOutOff = kQOff + kQBytes;           // staging: [16][512] fp32 (or bf16)
     static constexpr int kOutBytes = kOutRows * kDv * 4;
     // float [2][NG][4]: page maxima of the 4 lane quadrants, double-buffered
     // by page; the epilogue's row sums use the buffer of the item's last page.
@@ -209,7 +213,8 @@ struct FwdSmem {
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
     static_assert(kTmemUsed <= 512, "TMEM budget");
-    static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0, "swizzle atoms need 1 KB alignment");
+    static_assert(kQOff % 1024 == 0 && kStageBytes % 1024 == 0 && kPInStage % 1024 == 0,
+                  "swizzle atoms need 1 KB alignment");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -551,7 +556,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
     constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : NG == 32 ? kSwizzle64 : kSwizzle128;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
-    const uint32_t p_s = smem_addr(smem + L::kPOff);
+    const uint32_t p_s = kv_s + L::kPInStage;  // P^T of stage 0
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     WorkIter it;
     it.init(meta);
@@ -566,9 +571,8 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     while (ok && it.next(p, bginfo, item)) {
         for (int j = item.p0; j < item.p1; ++j) {
             const int st = s_it & 1;
-            const int pb = s_it % L::kPBuffers;
             const bool first = (j == item.p0);
-            ok = wait_bounded(bar0 + 8 * (kPFull0 + pb), (s_it / L::kPBuffers) & 1, ctl);
+            ok = wait_bounded(bar0 + 8 * (kPFull0 + st), (s_it >> 1) & 1, ctl);
             if (!ok) break;
             if (first) {
                 ok = wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl);
@@ -577,7 +581,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             MLA_TRACE_EV(kTrMmaPFull);
             tc_fence_after();
             const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
-            const uint64_t b_st = b_desc0 + ((pb * L::kPBytes) >> 4);
+            const uint64_t b_st = b_desc0 + ((st * L::kStageBytes) >> 4);
 #pragma unroll
             for (int k = 0; k < kPage / 16; ++k) {
                 const uint64_t b = b_st + ((k * 16 * NG * 2) >> 4);
@@ -590,7 +594,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             }
             issued = true;
             umma_commit(bar0 + 8 * (kKvEmpty0 + st));
-            umma_commit(bar0 + 8 * (kPEmpty0 + pb));
+            umma_commit(bar0 + 8 * (kPEmpty0 + st));
             MLA_TRACE_EV(kTrMmaG2Issued);
             ++s_it;
         }
@@ -610,7 +614,6 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     using Wp = FwdWarps<NG>;
     constexpr int NGW = Wp::kGroupCols;                   // query columns of this warp's group
     constexpr int W = NGW / 2;                            // own columns per thread
-    constexpr int kPB = L::kPBuffers;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int wq = warp & 3;                              // TMEM lane quadrant this warp may access
@@ -621,7 +624,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     const int gtg = gt & 127;                             // 0..127 within the column group
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
-    uint8_t* pbuf = smem + L::kPOff;
+    uint8_t* pbuf = smem + L::kKvOff + L::kPInStage;     // P^T of stage 0
     float* stage_f32 = reinterpret_cast<float*>(smem + L::kOutOff);
     __nv_bfloat16* stage_bf16 = reinterpret_cast<__nv_bfloat16*>(smem + L::kOutOff);
     // Token row of this thread in the page (M=64 accumulator: token m sits in
@@ -718,8 +721,8 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             float e[W];
 #pragma unroll
             for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
-            const int pb = s_it % kPB;
-            uint8_t* rowp = pbuf + pb * L::kPBytes + row * (NG * 2);
+            const int pb = s_it & 1;                      // the page's stage
+            uint8_t* rowp = pbuf + pb * L::kStageBytes + row * (NG * 2);
             auto store_p = [&](const float (&ev)[W]) {
                 uint32_t packed[W / 2];
 #pragma unroll
@@ -734,7 +737,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                         make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
                 }
             };
-            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it / kPB) & 1) ^ 1, ctl);
+            ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
             if (!ok) break;
             store_p(e);
             fence_proxy_async_smem();
@@ -786,7 +789,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     // GEMM2, then scale each of the group's columns (positions)
                     // in place.
                     const uint32_t prev = s_it - 1;
-                    ok = wait_warp(bar0 + 8 * (kPEmpty0 + prev % kPB), (prev / kPB) & 1, ctl);
+                    ok = wait_warp(bar0 + 8 * (kPEmpty0 + (prev & 1)), (prev >> 1) & 1, ctl);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
@@ -814,7 +817,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 
         // ---- epilogue: wait for the last GEMM2, reduce l over the tokens ----
         const uint32_t last = s_it - 1;
-        ok = wait_warp(bar0 + 8 * (kPEmpty0 + last % kPB), (last / kPB) & 1, ctl);
+        ok = wait_warp(bar0 + 8 * (kPEmpty0 + (last & 1)), (last >> 1) & 1, ctl);
         if (!ok) break;
         MLA_TRACE_SM(kTrSmEpi0);
         tc_fence_after();
