@@ -45,16 +45,22 @@ namespace mla {
 
 constexpr uint32_t kFullMask = 0xffffffffu;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-// Warps: TMA producer, kG1Issuers GEMM1 issuers, G2Issuers<NG> GEMM2 issuers,
+// Warps: TMA producer, G1<NG>::kIssuers GEMM1 issuers, G2Issuers<NG> GEMM2 issuers,
 // then the 4 softmax warps.  The softmax of NG = 32 needs more than the 224
 // registers per thread a ninth warp would leave, so it keeps one GEMM2 issuer.
 // A small tcgen05.mma (N <= 64, M = 64 or 128) occupies the tensor pipe for
 // about 50 cycles whatever its size, so the 52 MMAs of a 16-column page keep
-// the pipe busy for most of a page's HBM time.  Issued by two threads (warps 1
-// and 2, boxes alternating, each into its own accumulator) GEMM1 completes
-// ~15% sooner than from one thread in this kernel (bs16 x 64K: 214.5 vs
-// 247.3 us per launch, B200); per-box "landed" barriers did not help.
-constexpr int kG1Issuers = 2;
+// the pipe busy for most of a page's HBM time, and the page rate follows the
+// time GEMM1 and GEMM2 take to issue.  Issued from several threads (each into
+// its own accumulator) they complete sooner; measured on B200 at bs16 x 64K,
+// decode kernel per launch: GEMM1 from 1 / 2 / 3 threads 247.3 / 214.5 /
+// 204.3 us, and 4 GEMM2 threads (one per d_v chunk) with a one-page L2
+// prefetch 203.1 us.  32- and 64-column groups keep 2 + 1 issuers: their
+// softmax needs the registers a larger CTA would take away.
+template <int NG>
+struct G1 {
+    static constexpr int kIssuers = NG == 16 ? 3 : 2;  // GEMM1 issuer threads = S^T accumulators
+};
 // 64-column groups run 8 softmax warps: two column groups of 32 columns,
 // each the 4 warps that reach the four TMEM lane quadrants.  Their 384
 // threads leave 168 registers per thread at launch; warpgroup 0 (producer and
@@ -62,8 +68,8 @@ constexpr int kG1Issuers = 2;
 // warpgroups can hold the per-column state of 32 columns.
 template <int NG>
 struct FwdWarps {
-    static constexpr int kG2Issuers = NG == 16 ? 2 : 1;
-    static constexpr int kFirstG2 = 1 + kG1Issuers;
+    static constexpr int kG2Issuers = NG == 16 ? 4 : 1;
+    static constexpr int kFirstG2 = 1 + G1<NG>::kIssuers;
     static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
     static constexpr int kColGroups = NG == 64 ? 2 : 1;   // softmax column groups
     static constexpr int kGroupCols = NG / kColGroups;     // query columns per group
@@ -81,20 +87,16 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the running max gro
 constexpr float kLn2 = 0.693147180559945309f;
 // GEMM1 (S^T = K Q^T, K = 576) accumulates into one TMEM accumulator per
 // issuer; the softmax adds them.
-constexpr int kSChains = kG1Issuers;
 
 // L2 prefetch of whole pages ahead of the shared-memory loads
 // (cp.async.bulk.prefetch.L2, one 72 KB page per instruction).  With only two
-// 72 KB stages per SM the refill sees L2 rather than HBM latency (measured on
-// B200: ~1.7 us -> ~1.05 us per page at the bs16 x 64K load).  Short work
-// items gain nothing and lose a little, so only items of at least
+// 72 KB stages per SM the refill then sees L2 rather than HBM latency.
+// Measured on B200 at bs16 x 64K (decode kernel per launch): no prefetch
+// 228.9 us, 1 page ahead 212.5, 2 pages 214.6, 4 pages 218.5, 8 pages 271.7.
+// Short work items gain nothing and lose a little, so only items of at least
 // kPrefetchMinPages pages prefetch.
-#ifndef MLA_PREFETCH_PAGES
-#define MLA_PREFETCH_PAGES 2
-#endif
-constexpr int kPrefetchPages = MLA_PREFETCH_PAGES;
+constexpr int kPrefetchPages = 1;
 constexpr int kPrefetchMinPages = 16;
-static_assert(kSChains == kG1Issuers, "one S^T accumulator per GEMM1 issuer");
 
 // Optional timeline tracing (build with -DMLA_TRACE): each role of each CTA
 // stamps %globaltimer at pipeline events into a device buffer that the host
@@ -205,10 +207,10 @@ struct FwdSmem {
     // checks that the dynamic shared memory base is 1 KB aligned.
     static constexpr int kAlignSlack = kBytes + 1024 <= 227 * 1024 ? 1024 : 0;
     static constexpr int kAlloc = kBytes + kAlignSlack;
-    // TMEM columns: S^T buffer i, chain c at kSCol + (i*kSChains + c)*NG;
+    // TMEM columns: S^T buffer i, chain c at kSCol + (i*G1<NG>::kIssuers + c)*NG;
     // O^T d_v chunk c at kOCol + c*NG.
     static constexpr int kSCol = 0;
-    static constexpr int kOCol = 2 * kSChains * NG;
+    static constexpr int kOCol = 2 * G1<NG>::kIssuers * NG;
     static constexpr int kTmemUsed = kOCol + 4 * NG;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
@@ -515,11 +517,11 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
             if (!ok) break;
             tc_fence_after();
             // This issuer's accumulator; it takes boxes issuer, issuer + 2, ...
-            const uint32_t d = tmem + L::kSCol + (st * kSChains + issuer) * NG;
+            const uint32_t d = tmem + L::kSCol + (st * G1<NG>::kIssuers + issuer) * NG;
             const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
             bool first = true;
 #pragma unroll 1
-            for (int c = issuer; c < L::kBoxes; c += kG1Issuers) {
+            for (int c = issuer; c < L::kBoxes; c += G1<NG>::kIssuers) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const uint64_t a = a_st + ((c * L::kBoxBytes + k * 32) >> 4);
@@ -681,10 +683,10 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             tc_fence_after();
             float x[W];
             {
-                const uint32_t sbase = tmem + lane_base + L::kSCol + sb * kSChains * NG + c0g;
+                const uint32_t sbase = tmem + lane_base + L::kSCol + sb * G1<NG>::kIssuers * NG + c0g;
                 tmem_load_half<NGW>(sbase, x);
 #pragma unroll
-                for (int c = 1; c < kSChains; ++c) {
+                for (int c = 1; c < G1<NG>::kIssuers; ++c) {
                     float y[W];
                     tmem_load_half<NGW>(sbase + c * NG, y);
                     tmem_ld_wait();
@@ -1000,7 +1002,7 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
                 i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged)
                 count = FwdWarps<NG>::kSoftmaxThreads;
-            if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = kG1Issuers;
+            if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
             if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
                 count = FwdWarps<NG>::kG2Issuers;
             mbar_init(bar0 + 8 * i, count);
@@ -1026,7 +1028,7 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
                 prefetch_tensormap(&q_map);
                 run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
             }
-        } else if (warp <= kG1Issuers) {
+        } else if (warp <= G1<NG>::kIssuers) {
             if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
         } else {
             if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG>::kFirstG2);
