@@ -83,6 +83,16 @@ def test_workload_all_outputs(dev, name):
     print(name, m)
 
 
+def test_peaked_rows_on_few_ctas(dev):
+    """Peaked rows in long unsplit items: the running max is kept lazily, so a
+    dominant token's P need not be exactly 1; O is normalised by the sum of the
+    bf16 P it was accumulated with, which keeps these rows at the bf16 floor."""
+    d = workloads.make_inputs("b16_sq2_ragged1k16k_h16_peaked")
+    m = check(d, dev, num_sms=7)
+    print(m)
+    assert m["rmse"] <= m["q_floor"] + 5e-4
+
+
 def test_headline_sampled_outputs(dev):
     """batch 16 x 64K: the launch bench.py times, checked on sampled rows."""
     d = workloads.make_inputs("b16_l65536_h16")
