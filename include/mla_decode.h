@@ -72,6 +72,12 @@ extern "C" {
 
 /* dims.flags */
 #define MLA_FLAG_NO_COMBINE 0x1 /* mla_decode_fwd does not enqueue the combine; call mla_decode_combine */
+/* Test hook for the timeout path, never set in normal use: the producer of
+ * every CTA leaves the first page of its first work item unloaded, so the
+ * GEMM1 wait on it runs out after its 1 s limit.  The call then reports
+ * MLA_STATUS_TIMEOUT through mla_decode_get_status, its outputs are undefined,
+ * and the device stays usable. */
+#define MLA_FLAG_TEST_STALL 0x2
 
 typedef struct mla_decode_dims {
     int32_t batch;              /* B >= 1 */

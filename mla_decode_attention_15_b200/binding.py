@@ -30,6 +30,7 @@ MLA_STATUS_BAD_SCHEDULE = 0x8
 MLA_STATUS_SMEM_ALIGN = 0x10
 
 MLA_FLAG_NO_COMBINE = 0x1
+MLA_FLAG_TEST_STALL = 0x2
 
 PAGE_SIZE = 64
 D_QK = 576

@@ -164,6 +164,7 @@ struct FwdParams {
     int s_q, heads, N, num_blocks, max_blocks, causal;
     int G, BG, Hg, slots_cap;
     float scale_log2;  // softmax_scale * log2(e)
+    int test_stall;    // MLA_FLAG_TEST_STALL: leave the first page unloaded
 };
 
 struct CombineParams {
@@ -430,6 +431,8 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     it.init(meta);
     Item item;
     uint32_t kv_it = 0, q_it = 0;
+    uint32_t issued[2] = {0, 0};  // pages loaded per stage (for the abort drain)
+    bool stall = p.test_stall != 0;
     bool ok = true;
     MLA_TRACE_DECL(0);
     while (ok && it.next(p, bginfo, item)) {
@@ -459,6 +462,11 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
             const int st = kv_it & 1;
             ok = wait_bounded(bar0 + 8 * (kKvEmpty0 + st), ((kv_it >> 1) & 1) ^ 1, ctl);
             if (!ok) break;
+            if (stall) {  // test hook: this page is never loaded, so its GEMM1 wait runs out
+                stall = false;
+                ++kv_it;
+                continue;
+            }
             MLA_TRACE_EV(kTrProdIssue);
             int phys = __ldg(bt + j);
             if ((unsigned)phys >= (unsigned)p.num_blocks) {
@@ -471,15 +479,14 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
 #pragma unroll
             for (int c = 0; c < L::kBoxes; ++c)
                 tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, c * L::kBoxCols, 0, phys, policy);
+            ++issued[st];
             ++kv_it;
         }
     }
     if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        for (int st = 0; st < 2; ++st) {
-            const uint32_t n = (kv_it + 1 - st) / 2;
-            if (n > 0) wait_drain(bar0 + 8 * (kKvFull0 + st), (n - 1) & 1);
-        }
+        for (int st = 0; st < 2; ++st)
+            if (issued[st] > 0) wait_drain(bar0 + 8 * (kKvFull0 + st), (issued[st] - 1) & 1);
         if (q_it > 0) wait_drain(bar0 + 8 * kQFull, (q_it - 1) & 1);
     }
 }

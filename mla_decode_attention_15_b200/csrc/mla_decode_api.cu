@@ -24,7 +24,7 @@ int validate_dims(const mla_decode_dims* d) {
     if (d == nullptr) return MLA_ERR_INVALID_ARG;
     if (d->batch < 1 || d->s_q < 1 || d->num_heads < 1 || d->num_blocks < 1 ||
         d->max_blocks_per_seq < 1 || d->num_sms < 0 || d->reserved != 0 ||
-        (d->flags & ~MLA_FLAG_NO_COMBINE) != 0 || (d->causal != 0 && d->causal != 1))
+        (d->flags & ~(MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL)) != 0 || (d->causal != 0 && d->causal != 1))
         return MLA_ERR_INVALID_ARG;
     if (d->page_size != kPage || d->d_qk != kDqk || d->d_v != kDv) return MLA_ERR_UNSUPPORTED;
     if ((int64_t)d->num_heads * d->s_q > 256) return MLA_ERR_UNSUPPORTED;
@@ -361,6 +361,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.Hg = pl.gr.Hg;
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+    p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = pl.gr.NG == 16   ? launch_fwd<16>(pl, p, kvm, qm, st)
          : pl.gr.NG == 32 ? launch_fwd<32>(pl, p, kvm, qm, st)
