@@ -51,6 +51,9 @@ def parse_args():
                     help="decode only the first BATCH requests of the workload (small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="context/batch sweep (bs x L grid, 16 heads, s_q 1): one JSON line per point "
+                         "instead of the single bench line")
     return ap.parse_args()
 
 
@@ -538,8 +541,79 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
                     "copy) every step, inside one CUDA-graph replay per step, then a stream sync; KV cache resident"}
 
 
+SWEEP_BATCH = (1, 4, 8, 16, 32)
+SWEEP_LEN = (512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def run_sweep(args):
+    """Decode step and kernel time over a grid of batch x context length (16
+    heads, s_q 1, permuted pages, N(0,1) inputs).  The page pool is drawn on
+    the GPU; workloads whose KV fits in L2 are timed with an L2 flush between
+    steps.  One JSON line per grid point."""
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    bd.lib()
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, _, _ = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for B in SWEEP_BATCH:
+        for L in SWEEP_LEN:
+            d = workloads.build(B, 1, 16, ("fixed", L), seed=3000 + B, pool_device="cuda")
+            q, kv = d["q"].to(dev), d["kv_cache"]
+            bt, sl = d["block_table"].to(dev), d["cache_seqlens"].to(dev)
+            dims = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0)
+            dnc = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0, bd.MLA_FLAG_NO_COMBINE)
+            sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
+            ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+            out = torch.empty(B, 1, 16, 512, dtype=torch.bfloat16, device=dev)
+            lse = torch.empty(B, 16, 1, dtype=torch.float32, device=dev)
+            byt = algorithmic_bytes(d["cache_seqlens"], 1, 16)
+            use_flush = byt["total"] < (512 << 20)
+
+            def step(st, dm=dims):
+                bd.mla_decode_get_schedule(dm, sl, sched, st)
+                bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
+
+            times = []
+            for dm in (dims, dnc):
+                g = torch.cuda.CUDAGraph()
+                cap = torch.cuda.Stream()
+                cap.wait_stream(stream)
+                with torch.cuda.stream(cap):
+                    step(cap, dm)
+                    with torch.cuda.graph(g, stream=cap):
+                        step(cap, dm)
+                stream.wait_stream(cap)
+                ts = []
+                for i in range(3 + args.steps):
+                    if use_flush:
+                        flush.fill_(i & 255)
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    g.replay()
+                    b.record(stream)
+                    if i >= 3:
+                        ts.append((a, b))
+                torch.cuda.synchronize()
+                times.append(sum(x.elapsed_time(y) for x, y in ts) / len(ts))
+                del g
+            status = bd.mla_decode_get_status(sched)
+            ms_step, ms_kernel = times
+            print(json.dumps({"sweep": "context x batch", "batch": B, "kv_len": L, "heads": 16, "s_q": 1,
+                              "kv_bytes": byt["kv"], "us_per_call": ms_step * 1e3, "kernel_us": ms_kernel * 1e3,
+                              "kv_gbs": byt["kv"] / (ms_step * 1e-3) / 1e9,
+                              "kernel_frac_hbm": byt["total"] / (ms_kernel * 1e-3) / 1e9 / hbm_peak,
+                              "l2_flush": use_flush, "status": status}), flush=True)
+            del d, q, kv, bt, sl, sched, ws, out, lse
+            torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        return run_sweep(args)
     w = workloads.WORKLOADS[args.workload]
     if args.batch:
         import dataclasses

@@ -100,8 +100,13 @@ def _draw_lens(spec, batch: int, g: torch.Generator) -> torch.Tensor:
 
 def build(batch: int, s_q: int, heads: int, lens, sigma: float = 1.0, table: str = "permuted",
           peaked_frac: float = 0.0, seed: int = 0, spare_pages: int = 8,
-          tail_fill: Optional[float] = None, causal: bool = False) -> dict:
+          tail_fill: Optional[float] = None, causal: bool = False, pool_device: str = "cpu") -> dict:
     """Build one batch of decode inputs on the CPU.
+
+    ``pool_device`` other than "cpu" draws the page pool (step 3) there, from
+    a generator of that device seeded with ``seed + 1``, and leaves it there;
+    for multi-GB pools (sweeps, large-offset tests), whose oracle checks read
+    a host copy of it.  Every other draw stays on the CPU generator.
 
     ``lens`` is ("fixed", L), ("uniform", lo, hi) or ("list", [L_0, ...]).
     ``tail_fill`` (tests only) overwrites the rows past L_b in each request's
@@ -122,7 +127,12 @@ def build(batch: int, s_q: int, heads: int, lens, sigma: float = 1.0, table: str
     q = (torch.randn(batch * s_q * heads * D_QK, generator=g) * sigma).to(torch.bfloat16)
     q = q.view(batch, s_q, heads, D_QK)
     num_blocks = total_pages + spare_pages
-    kv = (torch.randn(num_blocks * PAGE * D_QK, generator=g) * sigma).to(torch.bfloat16)
+    if pool_device == "cpu":
+        kv = (torch.randn(num_blocks * PAGE * D_QK, generator=g) * sigma).to(torch.bfloat16)
+    else:
+        gd = torch.Generator(device=pool_device)
+        gd.manual_seed(int(seed) + 1)
+        kv = (torch.randn(num_blocks * PAGE * D_QK, generator=gd, device=pool_device) * sigma).to(torch.bfloat16)
     kv = kv.view(num_blocks, PAGE, 1, D_QK)
     if table == "identity":
         ids = torch.arange(num_blocks, dtype=torch.int32)

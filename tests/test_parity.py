@@ -105,6 +105,20 @@ def test_headline_sampled_outputs(dev):
     print(m)
 
 
+def test_pool_beyond_2gb_sampled_outputs(dev):
+    """bs16 x 128K: a 2.4 GB page pool, so most pages start past 2^31 bytes
+    (64-bit addressing of pages, TMA coordinates and output rows)."""
+    d = workloads.build(16, 1, 16, ("fixed", 131072), seed=2024, pool_device="cuda")
+    assert int(d["block_table"].max()) * 64 * 576 * 2 > 2 ** 31
+    out, lse, _ = run_gpu(d, dev)
+    rows = [0, 17, 90, 131, 170, 203, 250, 255]  # requests 0, 1, 5, 8, 10, 12, 15, 15
+    dh = dict(d)
+    dh["kv_cache"] = d["kv_cache"].cpu()
+    ro, rl = ref(dh, rows)
+    m = helpers.compare(out, lse, ro, rl, rows=rows)
+    print(m)
+
+
 def test_wide_heads_sampled_outputs(dev):
     """batch 32, s_q 2 causal, 128 heads (8 head groups of 32 columns)."""
     d = workloads.make_inputs("b32_sq2_ragged8k32k_h128")
