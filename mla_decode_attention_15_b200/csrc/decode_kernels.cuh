@@ -65,10 +65,13 @@ struct G1 {
 // each the 4 warps that reach the four TMEM lane quadrants.  Their 384
 // threads leave 168 registers per thread at launch; warpgroup 0 (producer and
 // issuers) gives registers back with setmaxnreg so that the softmax
-// warpgroups can hold the per-column state of 32 columns.
+// warpgroups can hold the per-column state of 32 columns.  (Measured on B200
+// at bs32 x s_q 2 x 128 heads: a 16-warp layout with 4 GEMM2 issuers and
+// 32-register issuers is slower, 648 vs 626 us per launch; a third GEMM1
+// accumulator does not fit TMEM at 64 columns.)
 template <int NG>
 struct FwdWarps {
-    static constexpr int kG2Issuers = NG == 16 ? 4 : 1;
+    static constexpr int kG2Issuers = NG == 16 ? 4 : 1;   // 4: one per d_v chunk
     static constexpr int kFirstG2 = 1 + G1<NG>::kIssuers;
     static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
     static constexpr int kColGroups = NG == 64 ? 2 : 1;   // softmax column groups
@@ -76,11 +79,12 @@ struct FwdWarps {
     static constexpr int kSoftmaxThreads = 128 * kColGroups;
     static constexpr int kThreads = 32 * kFirstSoftmax + kSoftmaxThreads;
     static constexpr bool kSplitRegs = NG == 64;
-    static constexpr int kRegsLaunch = 168;                 // 65536 / 384, rounded down to 8
+    static constexpr int kRegsLaunch = 65536 / kThreads / 8 * 8;
     static constexpr int kRegsIssue = 56;                   // warpgroup 0 after setmaxnreg.dec
     static constexpr int kRegsSoftmax = 224;                // softmax warpgroups after setmaxnreg.inc
-    static_assert(!kSplitRegs || (kFirstSoftmax == 4 && kThreads == 384), "warpgroup 0 = producer + issuers");
-    static_assert(!kSplitRegs || kRegsIssue * 128 + kRegsSoftmax * kSoftmaxThreads <= kRegsLaunch * kThreads,
+    static_assert(!kSplitRegs || kFirstSoftmax % 4 == 0, "setmaxnreg works on whole warpgroups");
+    static_assert(!kSplitRegs || kRegsIssue * 32 * kFirstSoftmax + kRegsSoftmax * kSoftmaxThreads <=
+                                     kRegsLaunch * kThreads,
                   "register split exceeds the launch allocation");
 };
 // Rescale O only when the running max grows by > 2^8.  Measured on B200
@@ -205,7 +209,8 @@ struct FwdSmem {
     // by page; the epilogue's row sums use the buffer of the item's last page.
     static constexpr int kRedOff = kOutOff + kOutBytes;
     static constexpr int kSumQOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]: sums of the bf16 P
-    static constexpr int kBarOff = kSumQOff + NG * 4 * 4;
+    static constexpr int kVoteOff = kSumQOff + NG * 4 * 4;     // uint32 [2][8]: per-warp growth votes
+    static constexpr int kBarOff = kVoteOff + 2 * 8 * 4;
     static constexpr int kNumBars = 24;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMiscOff + 16;
@@ -229,7 +234,7 @@ struct FwdSmem {
 enum Bar {
     kKvFull0 = 0, kKvFull1, kKvEmpty0, kKvEmpty1, kQFull, kQEmpty,
     kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
-    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kBarCount
+    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kMaxFull, kBarCount
 };
 static_assert(kBarCount <= FwdSmem<16>::kNumBars, "barrier slots");
 
@@ -431,7 +436,7 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     it.init(meta);
     Item item;
     uint32_t kv_it = 0, q_it = 0;
-    uint32_t issued[2] = {0, 0};  // pages loaded per stage (for the abort drain)
+    uint32_t issued0 = 0, issued1 = 0;  // pages loaded per stage (for the abort drain)
     bool stall = p.test_stall != 0;
     bool ok = true;
     MLA_TRACE_DECL(0);
@@ -479,14 +484,15 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
 #pragma unroll
             for (int c = 0; c < L::kBoxes; ++c)
                 tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, c * L::kBoxCols, 0, phys, policy);
-            ++issued[st];
+            issued0 += st == 0;
+            issued1 += st == 1;
             ++kv_it;
         }
     }
     if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        for (int st = 0; st < 2; ++st)
-            if (issued[st] > 0) wait_drain(bar0 + 8 * (kKvFull0 + st), (issued[st] - 1) & 1);
+        if (issued0 > 0) wait_drain(bar0 + 8 * kKvFull0, (issued0 - 1) & 1);
+        if (issued1 > 0) wait_drain(bar0 + 8 * kKvFull1, (issued1 - 1) & 1);
         if (q_it > 0) wait_drain(bar0 + 8 * kQFull, (q_it - 1) & 1);
     }
 }
@@ -638,6 +644,9 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     const int gtg = gt & 127;                             // 0..127 within the column group
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+    uint32_t* vote = reinterpret_cast<uint32_t*>(smem + L::kVoteOff);  // [2][softmax warps] growth flags
+    constexpr int kSoftmaxWarps = Wp::kSoftmaxThreads / 32;
+    const int sw = (threadIdx.x >> 5) - Wp::kFirstSoftmax;  // softmax warp index
     uint8_t* pbuf = smem + L::kKvOff + L::kPInStage;     // P^T of stage 0
     float* stage_f32 = reinterpret_cast<float*>(smem + L::kOutOff);
     __nv_bfloat16* stage_bf16 = reinterpret_cast<__nv_bfloat16*>(smem + L::kOutOff);
@@ -666,7 +675,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     WorkIter it;
     it.init(meta);
     Item item;
-    uint32_t s_it = 0, item_it = 0, out_it = 0;
+    uint32_t s_it = 0, item_it = 0, out_it = 0, max_it = 0;
     bool ok = true;
     while (ok && it.next(p, bginfo, item)) {
         int lvis[W];                                      // visible length of each own column
@@ -718,24 +727,36 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 #pragma unroll
             for (int i = 0; i < W; ++i) x[i] = (t < lvis[i]) ? x[i] * p.scale_log2 : -INFINITY;
 
-            // Page maxima of the own columns over the 16 tokens of this warp,
-            // then the four warps of the group meet through shared memory.
+            // Does any column's max grow by more than 2^8 on this page?
+            // 16/32-column groups: the warps post exact page maxima per column
+            // and meet once through shared memory.  64-column groups: each
+            // warp first posts only a one-word vote (any own value above the
+            // running max + 2^8); the maxima follow in a second round only if
+            // some warp voted.  That halves the common page's softmax work at
+            // 64 columns (B200, bs32 x s_q 2 x 128 heads: 626 -> 593 us per
+            // launch) but gains nothing at 16 and loses at 32 columns.
+            float m_own[W];
+#pragma unroll
+            for (int i = 0; i < W; ++i) m_own[i] = par ? m_all[2 * i + 1] : m_all[2 * i];
             float* rb = red + (s_it & 1) * NG * 4;
-            {
+            if constexpr (NG != 64) {
                 float xr[W];
 #pragma unroll
                 for (int i = 0; i < W; ++i) xr[i] = x[i];
                 const float wmax = HalfReduce<W, 0, true>::run(xr, lane);
                 if (red_w) rb[red_col * 4 + wq] = wmax;
+            } else {
+                bool grow_l = false;
+#pragma unroll
+                for (int i = 0; i < W; ++i) grow_l |= x[i] > m_own[i] + kRescaleLog2;
+                const uint32_t grow_w = __any_sync(kFullMask, grow_l) ? 1u : 0u;
+                if (lane == 0) vote[(s_it & 1) * kSoftmaxWarps + sw] = grow_w;
             }
             MLA_TRACE_SM(kTrSmMaxDone);
             mbar_arrive(bar0 + 8 * (kRedFull0 + (s_it & 1)));
 
             // Speculative P with the running max, stored before the exchange
-            // completes; it stands unless some column's max grows by > 2^8.
-            float m_own[W];
-#pragma unroll
-            for (int i = 0; i < W; ++i) m_own[i] = par ? m_all[2 * i + 1] : m_all[2 * i];
+            // completes; it stands unless some column's max grew by > 2^8.
             float e[W];
 #pragma unroll
             for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
@@ -764,26 +785,52 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             ok = wait_warp(bar0 + 8 * (kRedFull0 + (s_it & 1)), (s_it >> 1) & 1, ctl);
             if (!ok) break;
             MLA_TRACE_SM(kTrSmXchg);
-            bool grow = false;
+            bool grow_any = false;
+            if constexpr (NG != 64) {
+                // The warp's threads cover every column of the group and the
+                // group's four warps read the same maxima, so this decision is
+                // uniform across the group.
+                bool grow = false;
 #pragma unroll
-            for (int i = 0; i < W; ++i) {
-                const float4 r4 = *reinterpret_cast<const float4*>(rb + (c0g + par + 2 * i) * 4);
-                const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
-                grow |= pmax > m_own[i] + kRescaleLog2;
+                for (int i = 0; i < W; ++i) {
+                    const float4 r4 = *reinterpret_cast<const float4*>(rb + (c0g + par + 2 * i) * 4);
+                    const float pmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+                    grow |= pmax > m_own[i] + kRescaleLog2;
+                }
+                grow_any = __any_sync(kFullMask, grow);
+            } else {
+                // Every softmax warp reads every vote, so the decision is the
+                // same for all of them (the second round's barrier needs all).
+                uint32_t votes = 0;
+#pragma unroll
+                for (int w = 0; w < kSoftmaxWarps; w += 4) {
+                    const uint4 f4 = *reinterpret_cast<const uint4*>(vote + (s_it & 1) * kSoftmaxWarps + w);
+                    votes |= f4.x | f4.y | f4.z | f4.w;
+                }
+                grow_any = votes != 0;
+                if (grow_any) {
+                    float xr[W];
+#pragma unroll
+                    for (int i = 0; i < W; ++i) xr[i] = x[i];
+                    const float wmax = HalfReduce<W, 0, true>::run(xr, lane);
+                    if (red_w) rb[red_col * 4 + wq] = wmax;
+                    mbar_arrive(bar0 + 8 * kMaxFull);
+                    ok = wait_warp(bar0 + 8 * kMaxFull, max_it & 1, ctl);
+                    ++max_it;
+                    if (!ok) break;
+                }
             }
-            // The warp's threads cover every column of the group and the
-            // group's four warps read the same maxima, so this decision is
-            // uniform across the group.
-            if (!__any_sync(kFullMask, grow)) {
+            if (!grow_any) {
 #pragma unroll
                 for (int i = 0; i < W; ++i) {
                     l_own[i] += e[i];
                     lq_own[i] += bf16_round(e[i]);
                 }
             } else {
-                // Slow path (first page of an item, or a jump of the max):
-                // move the reference max of the grown columns, rescale.
+                // Slow path: the group's exact page maxima are in rb; move the
+                // reference max of the grown columns and rescale.
                 float alpha[NGW];
+                bool scale_any = false;
 #pragma unroll
                 for (int n = 0; n < NGW; ++n) {
                     const float4 r4 = *reinterpret_cast<const float4*>(rb + (c0g + n) * 4);
@@ -792,6 +839,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     if (mnew > m_all[n] + kRescaleLog2) {
                         alpha[n] = ex2_approx(m_all[n] - mnew);
                         m_all[n] = mnew;
+                        scale_any = true;
                     } else {
                         alpha[n] = 1.f;
                     }
@@ -804,9 +852,12 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     l_own[i] = l_own[i] * a + e[i];
                     lq_own[i] = lq_own[i] * a + bf16_round(e[i]);
                 }
-                store_p(e);
-                fence_proxy_async_smem();
-                if (j > item.p0) {
+                // scale_any is the same for the group's four warps (same maxima).
+                if (scale_any) {
+                    store_p(e);
+                    fence_proxy_async_smem();
+                }
+                if (scale_any && j > item.p0) {
                     // O^T already holds earlier pages: wait for the previous
                     // GEMM2, then scale each of the group's columns (positions)
                     // in place.
@@ -1027,7 +1078,7 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
         for (int i = 0; i < kBarCount; ++i) {
             uint32_t count = 1;
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
-                i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged)
+                i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged || i == kMaxFull)
                 count = FwdWarps<NG>::kSoftmaxThreads;
             if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
             if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
