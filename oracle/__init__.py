@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for absorbed-MQA MLA decode: TEST INFRASTRUCTURE.
+"""fp64 CPU oracle for absorbed-MQA MLA decode (and for the GQLA GQA path over
+a group-expanded cache, ``gqa_oracle_fwd``): TEST INFRASTRUCTURE.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
 arm of ``bench.py`` may import this package.  The product path (the CUDA
@@ -53,6 +54,15 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_longlong,
             ctypes.c_int,
+        ]
+        lib.gqa_oracle_fwd.restype = ctypes.c_int
+        lib.gqa_oracle_fwd.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
         ]
         lib.mla_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -127,4 +137,43 @@ def mla_oracle_fwd(q, kv, block_table, cache_seqlens, softmax_scale, causal=Fals
         raise RuntimeError("mla_oracle_fwd failed: %s (%d)" % (ERRORS.get(rc, "?"), rc))
     if want_probs:
         return out, lse, probs
+    return out, lse
+
+
+def gqa_oracle_fwd(q, kv, block_table, cache_seqlens, softmax_scale, groups, d_head=128, causal=False,
+                   rows=None, num_threads=0):
+    """Run the GQA-path oracle (see ``gqa_oracle_fwd`` in mla_oracle.c).
+
+    q: [B, s_q, h_q, d_head + d_rope]; kv: [num_blocks, page, (1,)
+    2*groups*d_head + d_rope]; both bf16 torch tensors or float64 arrays.
+    Returns (out [R, d_head] float64, lse [R] float64) for the flattened
+    query rows r = (b*s_q + s)*h_q + head, all of them or those in ``rows``.
+    """
+    lib = _load()
+    is_bf16 = isinstance(q, torch.Tensor) and q.dtype == torch.bfloat16
+    if isinstance(kv, torch.Tensor) and (kv.dtype == torch.bfloat16) != is_bf16:
+        raise TypeError("q and kv must both be bf16 or both be float64")
+    qn = _as_np(q, np.float64)
+    kvn = _as_np(kv, np.float64)
+    B, s_q, h, d_q = qn.shape
+    d_rope = d_q - d_head
+    num_blocks, page = kvn.shape[0], kvn.shape[1]
+    if d_rope < 0 or kvn.shape[-1] != 2 * groups * d_head + d_rope:
+        raise ValueError("kv row width must be 2*groups*d_head + d_rope")
+    bt = _as_np(block_table, np.int32).astype(np.int32)
+    sl = _as_np(cache_seqlens, np.int32).astype(np.int32)
+    if rows is None:
+        nrows, rows_np = B * s_q * h, None
+    else:
+        rows_np = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        nrows = rows_np.shape[0]
+    out = np.zeros((nrows, d_head), dtype=np.float64)
+    lse = np.zeros((nrows,), dtype=np.float64)
+    rc = lib.gqa_oracle_fwd(
+        B, s_q, h, int(groups), int(d_head), int(d_rope), page, int(bool(causal)), bt.shape[1], num_blocks,
+        qn.ctypes.data, kvn.ctypes.data, int(is_bf16), bt.ctypes.data, sl.ctypes.data,
+        float(softmax_scale), rows_np.ctypes.data if rows_np is not None else None, int(nrows),
+        out.ctypes.data, lse.ctypes.data, int(num_threads))
+    if rc != 0:
+        raise RuntimeError("gqa_oracle_fwd failed: %s (%d)" % (ERRORS.get(rc, "?"), rc))
     return out, lse

@@ -33,6 +33,9 @@
  * notes): the causal rule for s_q > 1 above; an empty visible range gives
  * O = 0 and LSE = -inf; no epsilon is added to l; LSE is the natural log.
  *
+ * The file also holds gqa_oracle_fwd (at the end): the GQLA "GQA path" over a
+ * group-expanded cache, pinned in tests/test_oracle_gqa.py.
+ *
  * Inputs are either fp64 arrays or bf16 bit patterns (uint16), converted to
  * double exactly.  Parallelism: OpenMP over query rows only; the arithmetic
  * inside a row is a plain sequential loop in token order.
@@ -168,4 +171,111 @@ int mla_oracle_max_threads(void) {
 #else
     return 1;
 #endif
+}
+
+/*
+ * GQA-path decode over a group-expanded cache, fp64 (GQLA technical summary,
+ * gist.science, pt, 2605.15250, section "Arquitetura", item 2 "Caminho GQA":
+ * the latent is expanded into g groups of keys and values, the cache keeps the
+ * per-group keys and values (2 g d_h per token) plus the shared RoPE key, and
+ * decode is standard grouped-query attention).  TEST INFRASTRUCTURE ONLY, like
+ * the rest of this file.
+ *
+ *   q      [batch][s_q][num_q_heads][d_head + d_rope]   (query head i, its
+ *          group part then its RoPE part)
+ *   kv     [num_blocks][page_size][2 * groups * d_head + d_rope]: per token
+ *          K_0 .. K_{g-1} (d_head each), V_0 .. V_{g-1} (d_head each), then
+ *          the shared RoPE key (d_rope)
+ *   head i belongs to group k = i / (num_q_heads / groups)
+ *   z_t  = scale * (<q_i[0:d_head], K_k[t]> + <q_i[d_head:], rope[t]>)
+ *   O_i  = sum_t softmax(z)_t * V_k[t]   (d_head wide),  LSE = m + log l
+ * with the same visible range and empty-range rule as mla_oracle_fwd.
+ * out [num_rows][d_head], lse [num_rows]; rows as in mla_oracle_fwd.
+ */
+int gqa_oracle_fwd(int batch, int s_q, int num_q_heads, int groups, int d_head, int d_rope,
+                   int page_size, int causal, int max_blocks_per_seq, long long num_blocks,
+                   const void* q, const void* kv, int inputs_are_bf16,
+                   const int32_t* block_table, const int32_t* cache_seqlens,
+                   double softmax_scale, const int32_t* rows, int num_rows,
+                   double* out, double* lse, int num_threads) {
+    if (batch < 0 || s_q < 1 || num_q_heads < 1 || groups < 1 || num_q_heads % groups != 0 ||
+        d_head < 1 || d_rope < 0 || page_size < 1 || max_blocks_per_seq < 0 || num_blocks < 0 || !q ||
+        !kv || !block_table || !cache_seqlens || !out || !lse)
+        return ORACLE_ERR_ARG;
+    const int d_q = d_head + d_rope;
+    const long long row_w = 2LL * groups * d_head + d_rope;
+    const int heads_per_group = num_q_heads / groups;
+    const long long total_rows = (long long)batch * s_q * num_q_heads;
+    long long nr = rows ? (long long)num_rows : total_rows;
+    if (rows) {
+        for (long long i = 0; i < nr; ++i)
+            if (rows[i] < 0 || rows[i] >= total_rows) return ORACLE_ERR_ARG;
+    }
+    for (int b = 0; b < batch; ++b) {
+        int L = cache_seqlens[b];
+        if (L < 0) return ORACLE_ERR_ARG;
+        long long pages = ((long long)L + page_size - 1) / page_size;
+        if (pages > max_blocks_per_seq) return ORACLE_ERR_BLOCK_TABLE;
+        for (long long j = 0; j < pages; ++j) {
+            int phys = block_table[(size_t)b * max_blocks_per_seq + j];
+            if (phys < 0 || phys >= num_blocks) return ORACLE_ERR_BLOCK_TABLE;
+        }
+    }
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#endif
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long i = 0; i < nr; ++i) {
+        long long r = rows ? rows[i] : i;
+        int h = (int)(r % num_q_heads);
+        int s = (int)((r / num_q_heads) % s_q);
+        int b = (int)(r / ((long long)num_q_heads * s_q));
+        int k = h / heads_per_group;
+        int L = cache_seqlens[b];
+        long long Lvis = (causal && s_q > 1) ? (long long)L - s_q + 1 + s : (long long)L;
+        if (Lvis < 0) Lvis = 0;
+        double* o = out + (size_t)i * d_head;
+        for (int c = 0; c < d_head; ++c) o[c] = 0.0;
+        if (Lvis == 0) {
+            lse[i] = -INFINITY;
+            continue;
+        }
+        double* z = (double*)malloc((size_t)Lvis * sizeof(double));
+        if (!z) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        const size_t q_off = (size_t)r * d_q;
+        const size_t k_col = (size_t)k * d_head;                            /* K_k */
+        const size_t v_col = (size_t)groups * d_head + (size_t)k * d_head;  /* V_k */
+        const size_t r_col = (size_t)2 * groups * d_head;                   /* shared RoPE key */
+        for (long long t = 0; t < Lvis; ++t) {
+            int phys = block_table[(size_t)b * max_blocks_per_seq + t / page_size];
+            size_t row_off = ((size_t)phys * page_size + (size_t)(t % page_size)) * (size_t)row_w;
+            double acc = 0.0;
+            for (int c = 0; c < d_head; ++c)
+                acc += load_elem(q, q_off + c, inputs_are_bf16) * load_elem(kv, row_off + k_col + c, inputs_are_bf16);
+            for (int c = 0; c < d_rope; ++c)
+                acc += load_elem(q, q_off + d_head + c, inputs_are_bf16) *
+                       load_elem(kv, row_off + r_col + c, inputs_are_bf16);
+            z[t] = softmax_scale * acc;
+        }
+        double m = z[0];
+        for (long long t = 1; t < Lvis; ++t)
+            if (z[t] > m) m = z[t];
+        double l = 0.0;
+        for (long long t = 0; t < Lvis; ++t) l += exp(z[t] - m);
+        for (long long t = 0; t < Lvis; ++t) {
+            int phys = block_table[(size_t)b * max_blocks_per_seq + t / page_size];
+            size_t row_off = ((size_t)phys * page_size + (size_t)(t % page_size)) * (size_t)row_w;
+            double w = exp(z[t] - m);
+            for (int c = 0; c < d_head; ++c) o[c] += w * load_elem(kv, row_off + v_col + c, inputs_are_bf16);
+        }
+        for (int c = 0; c < d_head; ++c) o[c] /= l;
+        lse[i] = m + log(l);
+        free(z);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
