@@ -183,6 +183,54 @@ int mla_decode_fwd_noalloc(const mla_decode_dims* dims, const void* q, const voi
                            const int32_t* block_table, const int32_t* cache_seqlens,
                            float softmax_scale, void* out, float* lse, void* stream);
 
+/* ------------------------------------------------------------------------
+ * GQA-path decode over a group-expanded cache (GQLA technical summary,
+ * gist.science, pt, 2605.15250, "Arquitetura", item 2 "Caminho GQA": the
+ * latent is expanded into g groups of keys and values; the cache keeps the
+ * per-group keys and values, 2 g d_h values per token, plus the shared RoPE
+ * key; decode is grouped-query attention).  Same transposed kernel as the
+ * MLA path (S^T = K Q^T, P^T = softmax over the KV axis, O^T = V^T P^T), with
+ * K = [K_g | RoPE] (192 wide) and V = V_g (128 wide) per group.
+ *
+ *   q            bf16 [batch][s_q][num_q_heads][192]: per head its 128-wide
+ *                group part, then its 64-wide RoPE part
+ *   kv_cache     bf16 [num_blocks][64][2 * num_kv_groups * 128 + 64]: per
+ *                token K_0 .. K_{g-1}, V_0 .. V_{g-1} (128 each), RoPE key (64)
+ *   block_table, cache_seqlens, causal rule: as for mla_decode_fwd
+ *   out          bf16 [batch][s_q][num_q_heads][128]
+ *   lse          fp32 [batch][num_q_heads][s_q] (natural log)
+ * Query head i reads group i / 16: num_q_heads must be 16 * num_kv_groups and
+ * s_q 1 or 2; d_head 128, d_rope 64, page_size 64 (else MLA_ERR_UNSUPPORTED).
+ * Errors, status word, schedule and workspace ownership, stream ordering and
+ * MLA_FLAG_* as for the mla_decode_* calls above; the schedule and workspace
+ * sizes come from the two _bytes calls below.  There is no allocation-free
+ * variant.  Each (request, KV group) is one work item of the split-KV plan.
+ * ---------------------------------------------------------------------- */
+typedef struct mla_gqa_dims {
+    int32_t batch;              /* B >= 1 */
+    int32_t s_q;                /* 1 or 2 */
+    int32_t num_q_heads;        /* 16 * num_kv_groups */
+    int32_t num_kv_groups;      /* g >= 1 */
+    int32_t num_blocks;         /* pages in the pool */
+    int32_t max_blocks_per_seq; /* row stride of block_table */
+    int32_t page_size;          /* must be 64 */
+    int32_t d_head;             /* must be 128 */
+    int32_t d_rope;             /* must be 64 */
+    int32_t causal;             /* as in mla_decode_dims */
+    int32_t num_sms;            /* persistent CTAs; 0 = the current device's SM count */
+    int32_t flags;              /* MLA_FLAG_* */
+} mla_gqa_dims;
+
+size_t mla_gqa_decode_schedule_bytes(const mla_gqa_dims* dims);
+size_t mla_gqa_decode_workspace_bytes(const mla_gqa_dims* dims);
+int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_seqlens, void* schedule,
+                                void* stream);
+int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* workspace, const void* q,
+                       const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
+                       float softmax_scale, void* out, float* lse, void* stream);
+int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,
+                           float* lse, void* stream);
+
 /* Library ABI version (increments on any change of these declarations). */
 int mla_decode_version(void);
 

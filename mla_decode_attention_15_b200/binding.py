@@ -47,7 +47,16 @@ EXPORTED = (
     "mla_decode_get_status",
     "mla_decode_strerror",
     "mla_decode_version",
+    "mla_gqa_decode_schedule_bytes",
+    "mla_gqa_decode_workspace_bytes",
+    "mla_gqa_decode_get_schedule",
+    "mla_gqa_decode_fwd",
+    "mla_gqa_decode_combine",
 )
+
+GQA_D_HEAD = 128
+GQA_D_ROPE = 64
+GQA_HEADS_PER_GROUP = 16
 
 
 class MlaDecodeError(RuntimeError):
@@ -60,6 +69,12 @@ class mla_decode_dims(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "batch", "s_q", "num_heads", "num_blocks", "max_blocks_per_seq", "page_size",
         "d_qk", "d_v", "causal", "num_sms", "flags", "reserved")]
+
+
+class mla_gqa_dims(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "batch", "s_q", "num_q_heads", "num_kv_groups", "num_blocks", "max_blocks_per_seq", "page_size",
+        "d_head", "d_rope", "causal", "num_sms", "flags")]
 
 
 _lib = None
@@ -99,6 +114,17 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_strerror.argtypes = [ctypes.c_int]
         L.mla_decode_version.restype = ctypes.c_int
         L.mla_decode_version.argtypes = []
+        Q = ctypes.POINTER(mla_gqa_dims)
+        L.mla_gqa_decode_schedule_bytes.restype = ctypes.c_size_t
+        L.mla_gqa_decode_schedule_bytes.argtypes = [Q]
+        L.mla_gqa_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.mla_gqa_decode_workspace_bytes.argtypes = [Q]
+        L.mla_gqa_decode_get_schedule.restype = ctypes.c_int
+        L.mla_gqa_decode_get_schedule.argtypes = [Q, vp, vp, vp]
+        L.mla_gqa_decode_fwd.restype = ctypes.c_int
+        L.mla_gqa_decode_fwd.argtypes = [Q, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+        L.mla_gqa_decode_combine.restype = ctypes.c_int
+        L.mla_gqa_decode_combine.argtypes = [Q, vp, vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -252,3 +278,94 @@ def mla_decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tenso
     dec.plan(cache_seqlens)
     out, lse = dec(q, kv_cache, block_table, cache_seqlens, softmax_scale)
     return out.clone(), lse.clone()
+
+
+# ---------------------------------------------------------------- GQA path
+def make_gqa_dims(batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
+                  causal: bool = False, num_sms: int = 0, flags: int = 0,
+                  num_q_heads: Optional[int] = None) -> mla_gqa_dims:
+    h = GQA_HEADS_PER_GROUP * num_kv_groups if num_q_heads is None else num_q_heads
+    return mla_gqa_dims(int(batch), int(s_q), int(h), int(num_kv_groups), int(num_blocks),
+                        int(max_blocks_per_seq), PAGE_SIZE, GQA_D_HEAD, GQA_D_ROPE, int(bool(causal)),
+                        int(num_sms), int(flags))
+
+
+def mla_gqa_decode_schedule_bytes(dims: mla_gqa_dims) -> int:
+    return int(lib().mla_gqa_decode_schedule_bytes(ctypes.byref(dims)))
+
+
+def mla_gqa_decode_workspace_bytes(dims: mla_gqa_dims) -> int:
+    return int(lib().mla_gqa_decode_workspace_bytes(ctypes.byref(dims)))
+
+
+def mla_gqa_decode_get_schedule(dims, cache_seqlens, schedule, stream=None) -> None:
+    _check(lib().mla_gqa_decode_get_schedule(ctypes.byref(dims), _ptr(cache_seqlens), _ptr(schedule),
+                                             _stream(stream)), "mla_gqa_decode_get_schedule")
+
+
+def mla_gqa_decode_fwd(dims, schedule, workspace, q, kv_cache, block_table, cache_seqlens,
+                       softmax_scale: float, out, lse, stream=None) -> None:
+    _check(lib().mla_gqa_decode_fwd(ctypes.byref(dims), _ptr(schedule), _ptr(workspace), _ptr(q),
+                                    _ptr(kv_cache), _ptr(block_table), _ptr(cache_seqlens),
+                                    float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_gqa_decode_fwd")
+
+
+def mla_gqa_decode_combine(dims, schedule, workspace, out, lse, stream=None) -> None:
+    _check(lib().mla_gqa_decode_combine(ctypes.byref(dims), _ptr(schedule), _ptr(workspace), _ptr(out),
+                                        _ptr(lse), _stream(stream)), "mla_gqa_decode_combine")
+
+
+class GqaDecoder:
+    """Schedule and workspace buffers for one shape of GQA-path decode batch
+    (group-expanded cache, 16 query heads per KV group); same use as
+    MlaDecoder."""
+
+    def __init__(self, batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
+                 causal: bool = False, num_sms: int = 0, device: Optional[torch.device] = None):
+        self.device = torch.device(device or "cuda")
+        if num_sms == 0:
+            num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        self.dims = make_gqa_dims(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq, causal, num_sms)
+        sb = mla_gqa_decode_schedule_bytes(self.dims)
+        wb = mla_gqa_decode_workspace_bytes(self.dims)
+        if sb == 0 or wb == 0:
+            raise MlaDecodeError(MLA_ERR_INVALID_ARG, "GqaDecoder dims")
+        h = self.dims.num_q_heads
+        self.row_width = 2 * num_kv_groups * GQA_D_HEAD + GQA_D_ROPE
+        self.schedule = torch.empty(sb, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.empty(wb, dtype=torch.uint8, device=self.device)
+        self.out = torch.empty(batch, s_q, h, GQA_D_HEAD, dtype=torch.bfloat16, device=self.device)
+        self.lse = torch.empty(batch, h, s_q, dtype=torch.float32, device=self.device)
+
+    def check_inputs(self, q, kv_cache, block_table, cache_seqlens) -> None:
+        d = self.dims
+        _require(q.dtype == torch.bfloat16 and q.is_contiguous() and
+                 tuple(q.shape) == (d.batch, d.s_q, d.num_q_heads, GQA_D_HEAD + GQA_D_ROPE),
+                 "q must be bf16 [B, s_q, 16*g, 192]")
+        _require(kv_cache.dtype == torch.bfloat16 and kv_cache.is_contiguous() and
+                 kv_cache.shape[0] == d.num_blocks and kv_cache.shape[1] == PAGE_SIZE and
+                 kv_cache.shape[-1] == self.row_width and
+                 kv_cache.numel() == d.num_blocks * PAGE_SIZE * self.row_width,
+                 "kv_cache must be bf16 [num_blocks, 64, 1, 2*g*128 + 64]")
+        _require(block_table.dtype == torch.int32 and block_table.is_contiguous() and
+                 tuple(block_table.shape) == (d.batch, d.max_blocks_per_seq),
+                 "block_table must be int32 [B, max_blocks_per_seq]")
+        _require(cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and
+                 tuple(cache_seqlens.shape) == (d.batch,), "cache_seqlens must be int32 [B]")
+        for t in (q, kv_cache, block_table, cache_seqlens):
+            _require(t.device == self.out.device, "all tensors must be on %s" % self.out.device)
+
+    def plan(self, cache_seqlens: torch.Tensor, stream=None) -> None:
+        mla_gqa_decode_get_schedule(self.dims, cache_seqlens, self.schedule, stream)
+
+    def __call__(self, q, kv_cache, block_table, cache_seqlens, softmax_scale: float,
+                 stream=None, check: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+        if check:
+            self.check_inputs(q, kv_cache, block_table, cache_seqlens)
+        mla_gqa_decode_fwd(self.dims, self.schedule, self.workspace, q, kv_cache, block_table,
+                           cache_seqlens, softmax_scale, self.out, self.lse, stream)
+        return self.out, self.lse
+
+    def status(self) -> int:
+        return mla_decode_get_status(self.schedule)

@@ -57,6 +57,43 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 // 204.3 us, and 4 GEMM2 threads (one per d_v chunk) with a one-page L2
 // prefetch 203.1 us.  32- and 64-column groups keep 2 + 1 issuers: their
 // softmax needs the registers a larger CTA would take away.
+// Cache shapes.  ShapeMla (absorbed MQA, the main path): a 576-wide row
+// (512 latent + 64 RoPE) is the key and its first 512 columns the value.
+// ShapeGqa (the GQLA summary's "Caminho GQA"): per token, g groups of
+// 128-wide keys, then g groups of 128-wide values, then one shared 64-wide
+// RoPE key; a work item reads its group's key (2 boxes of 64 columns), the
+// RoPE key and its group's value.  Stage box kRopeBox is read by GEMM1 only,
+// so the softmax writes the page's P^T over it.
+struct ShapeMla {
+    static constexpr int kDqk = 576, kDv = 512;
+    static constexpr int kKBoxes = 9;      // K (and Q) boxes of 64 columns
+    static constexpr int kStageBoxes = 9;  // boxes loaded per page
+    static constexpr int kRopeBox = 8;
+    static constexpr int kVChunks = 4;     // d_v / 128: GEMM2 chunks of 128 rows
+    static constexpr bool kPrefetchL2 = true;  // a page is one contiguous 72 KB block
+    __host__ __device__ static constexpr int k_box(int c) { return c; }
+    // first stage box of d_v chunk ch; the chunk's second box follows 8 KB on
+    __host__ __device__ static constexpr int v_box(int ch) { return 2 * ch; }
+    // cache column of stage box c for KV group kg of kv_groups
+    __host__ __device__ static constexpr int col(int c, int, int) { return 64 * c; }
+    __host__ __device__ static constexpr int row_width(int) { return kDqk; }
+};
+struct ShapeGqa {
+    static constexpr int kDh = 128, kDrope = 64;
+    static constexpr int kDqk = kDh + kDrope, kDv = kDh;
+    static constexpr int kKBoxes = 3;      // K_g (2 boxes) + the RoPE key
+    static constexpr int kStageBoxes = 5;  // K_g, K_g, RoPE, V_g, V_g
+    static constexpr int kRopeBox = 2;
+    static constexpr int kVChunks = 1;
+    static constexpr bool kPrefetchL2 = false;  // a group's boxes are strided across the page
+    __host__ __device__ static constexpr int k_box(int c) { return c; }
+    __host__ __device__ static constexpr int v_box(int) { return 3; }
+    __host__ __device__ static constexpr int col(int c, int kg, int kv_groups) {
+        return c < 2 ? kg * kDh + 64 * c : c == 2 ? 2 * kv_groups * kDh : kv_groups * kDh + kg * kDh + 64 * (c - 3);
+    }
+    __host__ __device__ static constexpr int row_width(int kv_groups) { return 2 * kv_groups * kDh + kDrope; }
+};
+
 template <int NG>
 struct G1 {
     static constexpr int kIssuers = NG == 16 ? 3 : 2;  // GEMM1 issuer threads = S^T accumulators
@@ -69,9 +106,9 @@ struct G1 {
 // at bs32 x s_q 2 x 128 heads: a 16-warp layout with 4 GEMM2 issuers and
 // 32-register issuers is slower, 648 vs 626 us per launch; a third GEMM1
 // accumulator does not fit TMEM at 64 columns.)
-template <int NG>
+template <int NG, class S = ShapeMla>
 struct FwdWarps {
-    static constexpr int kG2Issuers = NG == 16 ? 4 : 1;   // 4: one per d_v chunk
+    static constexpr int kG2Issuers = NG == 16 && S::kVChunks >= 4 ? 4 : 1;  // 4: one per d_v chunk
     static constexpr int kFirstG2 = 1 + G1<NG>::kIssuers;
     static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
     static constexpr int kColGroups = NG == 64 ? 2 : 1;   // softmax column groups
@@ -169,7 +206,16 @@ struct FwdParams {
     int G, BG, Hg, slots_cap;
     float scale_log2;  // softmax_scale * log2(e)
     int test_stall;    // MLA_FLAG_TEST_STALL: leave the first page unloaded
+    // Query columns of a work item: runs of run_rows consecutive rows, run r
+    // at row offset r * run_stride + g * run_rows (one run for MLA groups;
+    // one run per new token for GQA groups).  kv_groups: GQA groups.
+    int run_rows, run_stride, kv_groups;
 };
+// Query column (in [0, N)) of column q of group g.
+__device__ __forceinline__ int item_col(int run_rows, int run_stride, int g, int q) {
+    const int r = q / run_rows;
+    return r * run_stride + g * run_rows + (q - r * run_rows);
+}
 
 struct CombineParams {
     const int32_t* sched;
@@ -179,32 +225,33 @@ struct CombineParams {
     float* lse;
     int32_t* status;
     int s_q, heads, N, NG, Hg, G, BG, slots_cap;
+    int run_rows, run_stride;
 };
 
 // ------------------------------------------------------------------ layout
-template <int NG>
+template <int NG, class S = ShapeMla>
 struct FwdSmem {
     static constexpr int kStages = 2;
     static constexpr int kBoxCols = 64;
     static constexpr int kBoxBytes = kPage * kBoxCols * 2;    // 8 KB: 64 tokens x 64 cols
-    static constexpr int kBoxes = kDqk / kBoxCols;            // 9
-    static constexpr int kStageBytes = kBoxes * kBoxBytes;    // 72 KB: one page
+    static constexpr int kBoxes = S::kStageBoxes;             // boxes per page (9 for MLA)
+    static constexpr int kStageBytes = kBoxes * kBoxBytes;    // 72 KB: one MLA page
     static constexpr int kQBoxBytes = NG * 128;               // NG rows x 64 cols
-    static constexpr int kQBytes = kBoxes * kQBoxBytes;
+    static constexpr int kQBytes = S::kKBoxes * kQBoxBytes;
     static constexpr int kPBytes = kPage * NG * 2;            // P^T of one page, bf16
     // P^T of a page is written over the page's own RoPE box (box 8): only
     // GEMM1 reads that box, S^T is complete before the softmax writes P^T, and
     // the stage is refilled only after the page's GEMM2 has read P^T.  So P^T
     // is double-buffered with the stages at no cost in shared memory.
-    static constexpr int kPInStage = 8 * kBoxBytes;
+    static constexpr int kPInStage = S::kRopeBox * kBoxBytes;
     static_assert(kPBytes <= kBoxBytes, "P^T fits the RoPE box");
     static constexpr int kKvOff = 0;
     static constexpr int kQOff = kKvOff + kStages * kStageBytes;
     // 64-column groups: Q^T takes 72 KB, so the epilogue stores straight from
     // registers (no staging tile).
     static constexpr int kOutRows = NG == 64 ? 0 : 16;        // output rows (query columns) per staging pass
-    static constexpr int kOutOff = kQOff + kQBytes;           // staging: [16][512] fp32 (or bf16)
-    static constexpr int kOutBytes = kOutRows * kDv * 4;
+    static constexpr int kOutOff = kQOff + kQBytes;           // staging: [16][d_v] fp32 (or bf16)
+    static constexpr int kOutBytes = kOutRows * S::kDv * 4;
     // float [2][NG][4]: page maxima of the 4 lane quadrants, double-buffered
     // by page; the epilogue's row sums use the buffer of the item's last page.
     static constexpr int kRedOff = kOutOff + kOutBytes;
@@ -222,7 +269,7 @@ struct FwdSmem {
     // O^T d_v chunk c at kOCol + c*NG.
     static constexpr int kSCol = 0;
     static constexpr int kOCol = 2 * G1<NG>::kIssuers * NG;
-    static constexpr int kTmemUsed = kOCol + 4 * NG;
+    static constexpr int kTmemUsed = kOCol + S::kVChunks * NG;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
     static_assert(kTmemUsed <= 512, "TMEM budget");
@@ -423,11 +470,11 @@ __device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const float (&v)
 }
 
 // ------------------------------------------------------------------ roles
-template <int NG>
+template <int NG, class S>
 __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map,
                              const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                              uint8_t* smem, const Ctl& ctl) {
-    using L = FwdSmem<NG>;
+    using L = FwdSmem<NG, S>;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t q_s = smem_addr(smem + L::kQOff);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
@@ -445,13 +492,17 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
         ok = wait_bounded(bar0 + 8 * kQEmpty, (q_it & 1) ^ 1, ctl);
         if (!ok) break;
         mbar_arrive_expect_tx(bar0 + 8 * kQFull, L::kQBytes);
-        const int row0 = item.b * p.N + item.g * NG;
 #pragma unroll 1
-        for (int c = 0; c < L::kBoxes; ++c)
-            tma_load_2d(q_s + c * L::kQBoxBytes, q_map, bar0 + 8 * kQFull, c * L::kBoxCols, row0);
+        for (int r = 0; r * p.run_rows < NG; ++r) {  // runs of query rows (one for MLA groups)
+            const int row0 = item.b * p.N + r * p.run_stride + item.g * p.run_rows;
+#pragma unroll 1
+            for (int c = 0; c < S::kKBoxes; ++c)
+                tma_load_2d(q_s + c * L::kQBoxBytes + r * p.run_rows * 128, q_map, bar0 + 8 * kQFull,
+                            c * L::kBoxCols, row0);
+        }
         ++q_it;
         const int32_t* bt = p.block_table + (size_t)item.b * p.max_blocks;
-        const bool prefetch = kPrefetchPages > 0 && item.p1 - item.p0 >= kPrefetchMinPages;
+        const bool prefetch = S::kPrefetchL2 && kPrefetchPages > 0 && item.p1 - item.p0 >= kPrefetchMinPages;
         if (prefetch)
             for (int j = item.p0; j < item.p1 && j < item.p0 + kPrefetchPages; ++j) {
                 const int ph = __ldg(bt + j);
@@ -483,7 +534,8 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
             const uint32_t dst = kv_s + st * L::kStageBytes;
 #pragma unroll
             for (int c = 0; c < L::kBoxes; ++c)
-                tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, c * L::kBoxCols, 0, phys, policy);
+                tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, S::col(c, item.g, p.kv_groups), 0, phys,
+                                 policy);
             issued0 += st == 0;
             issued1 += st == 1;
             ++kv_it;
@@ -502,10 +554,10 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
 // 8-row groups 1 KB apart) and K-major B (Q^T rows); the 16-wide k-step
 // advances 32 B inside the 128-byte swizzle atom.  k-step i accumulates into
 // the accumulator of its issuer.
-template <int NG>
+template <int NG, class S>
 __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                           uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
-    using L = FwdSmem<NG>;
+    using L = FwdSmem<NG, S>;
     constexpr uint32_t kIdescS = idesc_bf16_f32(64, NG, 0, 0);
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t q_s = smem_addr(smem + L::kQOff);
@@ -539,10 +591,10 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
             const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
             bool first = true;
 #pragma unroll 1
-            for (int c = issuer; c < L::kBoxes; c += G1<NG>::kIssuers) {
+            for (int c = issuer; c < S::kKBoxes; c += G1<NG>::kIssuers) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint64_t a = a_st + ((c * L::kBoxBytes + k * 32) >> 4);
+                    const uint64_t a = a_st + ((S::k_box(c) * L::kBoxBytes + k * 32) >> 4);
                     const uint64_t b = b_desc0 + ((c * L::kQBoxBytes + k * 32) >> 4);
                     umma_f16(d, a, b, kIdescS, first ? 0u : 1u);
                     first = false;
@@ -567,12 +619,12 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
 // contiguous within a token row; 64 d_v per swizzle atom, next atom = next box
 // 8 KB on, 8-token groups 1 KB apart); P^T is MN-major with NG columns per
 // token row.  k-outer order keeps consecutive MMAs on different accumulators.
-template <int NG>
+template <int NG, class S>
 __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                           uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
-    constexpr int kIssuers = FwdWarps<NG>::kG2Issuers;
-    constexpr int kChunksPer = (kDv / 128) / kIssuers;  // d_v chunks of 128 per issuer
-    using L = FwdSmem<NG>;
+    constexpr int kIssuers = FwdWarps<NG, S>::kG2Issuers;
+    constexpr int kChunksPer = S::kVChunks / kIssuers;  // d_v chunks of 128 per issuer
+    using L = FwdSmem<NG, S>;
     constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
     constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : NG == 32 ? kSwizzle64 : kSwizzle128;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
@@ -608,7 +660,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
 #pragma unroll
                 for (int cc = 0; cc < kChunksPer; ++cc) {
                     const int ch = issuer * kChunksPer + cc;
-                    const uint64_t a = a_st + (((2 * ch) * L::kBoxBytes + k * 2048) >> 4);
+                    const uint64_t a = a_st + ((S::v_box(ch) * L::kBoxBytes + k * 2048) >> 4);
                     umma_f16(tmem + L::kOCol + ch * NG, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
                 }
             }
@@ -627,11 +679,11 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     }
 }
 
-template <int NG>
+template <int NG, class S>
 __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
                             uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
-    using L = FwdSmem<NG>;
-    using Wp = FwdWarps<NG>;
+    using L = FwdSmem<NG, S>;
+    using Wp = FwdWarps<NG, S>;
     constexpr int NGW = Wp::kGroupCols;                   // query columns of this warp's group
     constexpr int W = NGW / 2;                            // own columns per thread
     const int warp = threadIdx.x >> 5;
@@ -681,7 +733,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         int lvis[W];                                      // visible length of each own column
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-            const int gc = item.g * NG + c0g + par + 2 * i;
+            const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + par + 2 * i);
             int v = 0;
             if (gc < p.N) {
                 const int sq = gc / p.heads;
@@ -866,7 +918,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
-                    for (int ch = 0; ch < kDv / 128; ++ch) {
+                    for (int ch = 0; ch < S::kVChunks; ++ch) {
 #pragma unroll
                         for (int h = 0; h < NGW; h += 16) {  // 16 positions at a time
                             float o[16];
@@ -932,7 +984,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             l_gt = gtg == n ? ls : l_gt;
         }
         {
-            const int gc = item.g * NG + c0g + gtg;
+            const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + gtg);
             if (gtg < NGW && gc < p.N) {
                 const float lse = l_gt > 0.f ? (m_gt + log2f(l_gt)) * kLn2 : -INFINITY;
                 if (item.unsplit) {
@@ -956,7 +1008,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 if (!ok) break;
                 const bool f32 = !item.unsplit;
 #pragma unroll 1
-                for (int ch = 0; ch < kDv / 128; ++ch) {
+                for (int ch = 0; ch < S::kVChunks; ++ch) {
                     // positions 8ps.. hold even columns 16ps + 2i, NG/2 + 8ps.. the odd ones
                     float ev[8], od[8];
                     const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
@@ -969,11 +1021,11 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                         const float ve = ev[i] * inv[16 * ps + 2 * i];
                         const float vo = od[i] * inv[16 * ps + 2 * i + 1];
                         if (f32) {
-                            stage_f32[(2 * i) * kDv + d] = ve;
-                            stage_f32[(2 * i + 1) * kDv + d] = vo;
+                            stage_f32[(2 * i) * S::kDv + d] = ve;
+                            stage_f32[(2 * i + 1) * S::kDv + d] = vo;
                         } else {
-                            stage_bf16[(2 * i) * kDv + d] = __float2bfloat16_rn(ve);
-                            stage_bf16[(2 * i + 1) * kDv + d] = __float2bfloat16_rn(vo);
+                            stage_bf16[(2 * i) * S::kDv + d] = __float2bfloat16_rn(ve);
+                            stage_bf16[(2 * i + 1) * S::kDv + d] = __float2bfloat16_rn(vo);
                         }
                     }
                 }
@@ -982,17 +1034,18 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                 if (gt == 0) {
                     ok = wait_bounded(bar0 + 8 * kOutStaged, out_it & 1, ctl);
                     if (ok) {
-                        const int c0 = item.g * NG + L::kOutRows * ps;  // first query column of the pass
+                        // first query column of the pass; a pass stays within one run
+                        const int c0 = item_col(p.run_rows, p.run_stride, item.g, L::kOutRows * ps);
                         if (f32) {
                             if (item.slot >= 0)
-                                bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * kDv,
-                                               smem_addr(stage_f32), L::kOutRows * kDv * 4);
+                                bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * S::kDv,
+                                               smem_addr(stage_f32), L::kOutRows * S::kDv * 4);
                         } else {
                             int rows = p.N - c0;
                             rows = rows < L::kOutRows ? rows : L::kOutRows;
                             if (rows > 0)
-                                bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * kDv, smem_addr(stage_bf16),
-                                               rows * kDv * 2);
+                                bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * S::kDv, smem_addr(stage_bf16),
+                                               rows * S::kDv * 2);
                         }
                         bulk_commit();
                         bulk_wait_read_all();
@@ -1009,7 +1062,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             // bytes.
             const bool f32 = !item.unsplit;
 #pragma unroll 1
-            for (int ch = 0; ch < kDv / 128; ++ch) {
+            for (int ch = 0; ch < S::kVChunks; ++ch) {
 #pragma unroll
               for (int h = 0; h < NGW; h += 16) {  // 16 positions at a time
                 float o[16];
@@ -1021,10 +1074,10 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     const int n = pos_to_col(h + q, NGW);          // group column of position h + q
                     const float v = o[q] * inv[n];
                     if (f32) {
-                        if (item.slot >= 0) p.opart[((size_t)item.slot * NG + c0g + n) * kDv + d] = v;
+                        if (item.slot >= 0) p.opart[((size_t)item.slot * NG + c0g + n) * S::kDv + d] = v;
                     } else {
-                        const int gc = item.g * NG + c0g + n;
-                        if (gc < p.N) p.out[((size_t)item.b * p.N + gc) * kDv + d] = __float2bfloat16_rn(v);
+                        const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + n);
+                        if (gc < p.N) p.out[((size_t)item.b * p.N + gc) * S::kDv + d] = __float2bfloat16_rn(v);
                     }
                 }
               }
@@ -1042,11 +1095,11 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 }
 
 // ------------------------------------------------------------------ kernels
-template <int NG>
-__global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
+template <int NG, class S>
+__global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
     mla_decode_fwd_kernel(const __grid_constant__ CUtensorMap kv_map,
                           const __grid_constant__ CUtensorMap q_map, const FwdParams p) {
-    using L = FwdSmem<NG>;
+    using L = FwdSmem<NG, S>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -1079,10 +1132,10 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
             uint32_t count = 1;
             if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
                 i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged || i == kMaxFull)
-                count = FwdWarps<NG>::kSoftmaxThreads;
+                count = FwdWarps<NG, S>::kSoftmaxThreads;
             if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
             if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
-                count = FwdWarps<NG>::kG2Issuers;
+                count = FwdWarps<NG, S>::kG2Issuers;
             mbar_init(bar0 + 8 * i, count);
         }
         *abort_flag = 0;
@@ -1098,22 +1151,22 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const Ctl ctl{abort_flag, p.status};
 
-    if (warp < FwdWarps<NG>::kFirstSoftmax) {
-        if constexpr (FwdWarps<NG>::kSplitRegs) setmaxnreg_dec<FwdWarps<NG>::kRegsIssue>();
+    if (warp < FwdWarps<NG, S>::kFirstSoftmax) {
+        if constexpr (FwdWarps<NG, S>::kSplitRegs) setmaxnreg_dec<FwdWarps<NG, S>::kRegsIssue>();
         if (warp == 0) {
             if (lane == 0) {
                 prefetch_tensormap(&kv_map);
                 prefetch_tensormap(&q_map);
-                run_producer<NG>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
+                run_producer<NG, S>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
             }
         } else if (warp <= G1<NG>::kIssuers) {
-            if (lane == 0) run_gemm1<NG>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
+            if (lane == 0) run_gemm1<NG, S>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
         } else {
-            if (lane == 0) run_gemm2<NG>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG>::kFirstG2);
+            if (lane == 0) run_gemm2<NG, S>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG, S>::kFirstG2);
         }
     } else {
-        if constexpr (FwdWarps<NG>::kSplitRegs) setmaxnreg_inc<FwdWarps<NG>::kRegsSoftmax>();
-        run_softmax<NG>(p, meta, bginfo, smem, tmem, ctl);
+        if constexpr (FwdWarps<NG, S>::kSplitRegs) setmaxnreg_inc<FwdWarps<NG, S>::kRegsSoftmax>();
+        run_softmax<NG, S>(p, meta, bginfo, smem, tmem, ctl);
     }
     tc_fence_before();
     __syncthreads();
@@ -1128,11 +1181,10 @@ __global__ void __launch_bounds__(FwdWarps<NG>::kThreads, 1)
 // merge is one round of loads: the k partial LSEs are read one per thread and
 // reduced across the block while the first kCombinePre partial rows are
 // already in flight; further rows are read kCombineUnroll at a time.
-constexpr int kCombineThreads = kDv / 4;
 constexpr int kCombinePre = 8;
 constexpr int kCombineUnroll = 8;
 
-template <bool kMax>
+template <int kCombineThreads, bool kMax>
 __device__ __forceinline__ float combine_block_reduce(float v, float* red) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -1155,7 +1207,9 @@ __device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
     acc.w = fmaf(w, v.w, acc.w);
 }
 
-__global__ void __launch_bounds__(kCombineThreads) mla_decode_combine_kernel(const CombineParams p) {
+template <int kDv>
+__global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const CombineParams p) {
+    constexpr int kCombineThreads = kDv / 4;
     __shared__ float red[kCombineThreads / 32];
     __shared__ float wts[kCombineThreads];
     const int bg = blockIdx.x;
@@ -1170,7 +1224,7 @@ __global__ void __launch_bounds__(kCombineThreads) mla_decode_combine_kernel(con
     }
     const int b = bg / p.Hg;
     const int g = bg - b * p.Hg;
-    const int gc = g * p.NG + n;
+    const int gc = item_col(p.run_rows, p.run_stride, g, n);
     if (gc >= p.N) return;
     const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
     const int base = __ldg(info + 0);
@@ -1198,12 +1252,12 @@ __global__ void __launch_bounds__(kCombineThreads) mla_decode_combine_kernel(con
         float mx = own;
         for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads)
             mx = fmaxf(mx, __ldg(lp + (size_t)i * p.NG));
-        mx = combine_block_reduce<true>(mx, red);
+        mx = combine_block_reduce<kCombineThreads, true>(mx, red);
         if (mx != -INFINITY) {  // uniform across the block
             float sum = 0.f;
             for (int i = threadIdx.x; i < k; i += kCombineThreads)
                 sum += expf((i == threadIdx.x ? own : __ldg(lp + (size_t)i * p.NG)) - mx);
-            sum = combine_block_reduce<false>(sum, red);
+            sum = combine_block_reduce<kCombineThreads, false>(sum, red);
             lstar = mx + logf(sum);
             for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
                 const int cn = k - c0 < kCombineThreads ? k - c0 : kCombineThreads;

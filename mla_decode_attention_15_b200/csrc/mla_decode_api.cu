@@ -17,7 +17,7 @@ namespace {
 
 using namespace mla;
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int kMaxDevices = 64;
 
 int validate_dims(const mla_decode_dims* d) {
@@ -75,9 +75,43 @@ int make_plan(const mla_decode_dims* d, Plan* pl) {
     return MLA_OK;
 }
 
-size_t workspace_bytes_of(const Plan& pl) {
-    const size_t per_slot = (size_t)pl.gr.NG * (kDv + 1) * sizeof(float);
+size_t workspace_bytes_of(const Plan& pl, int d_v = kDv) {
+    const size_t per_slot = (size_t)pl.gr.NG * (d_v + 1) * sizeof(float);
     return (size_t)pl.slots * per_slot;
+}
+
+// ---- GQA path: groups of 16 query heads x s_q new tokens, one per KV group ----
+constexpr int kGqaHeadsPerGroup = 16;
+
+int validate_gqa(const mla_gqa_dims* d) {
+    if (d == nullptr) return MLA_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->s_q < 1 || d->num_q_heads < 1 || d->num_kv_groups < 1 || d->num_blocks < 1 ||
+        d->max_blocks_per_seq < 1 || d->num_sms < 0 ||
+        (d->flags & ~(MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL)) != 0 || (d->causal != 0 && d->causal != 1))
+        return MLA_ERR_INVALID_ARG;
+    if (d->page_size != kPage || d->d_head != ShapeGqa::kDh || d->d_rope != ShapeGqa::kDrope || d->s_q > 2 ||
+        (int64_t)d->num_q_heads != (int64_t)kGqaHeadsPerGroup * d->num_kv_groups || d->num_kv_groups > 64)
+        return MLA_ERR_UNSUPPORTED;
+    const int64_t BG = (int64_t)d->batch * d->num_kv_groups;
+    if (BG * ((int64_t)d->max_blocks_per_seq + kItemOverhead) >= (int64_t)INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * d->num_q_heads * d->s_q >= (int64_t)INT32_MAX / 2) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * d->max_blocks_per_seq >= (int64_t)INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+int make_plan_gqa(const mla_gqa_dims* d, Plan* pl) {
+    int rc = validate_gqa(d);
+    if (rc != MLA_OK) return rc;
+    mla_decode_dims tmp = {};
+    tmp.num_sms = d->num_sms;
+    rc = resolve_ctas(&tmp, &pl->G);
+    if (rc != MLA_OK) return rc;
+    pl->gr.N = d->num_q_heads * d->s_q;
+    pl->gr.NG = kGqaHeadsPerGroup * d->s_q;
+    pl->gr.Hg = d->num_kv_groups;
+    pl->BG = d->batch * d->num_kv_groups;
+    pl->slots = max_slots(pl->G);
+    return MLA_OK;
 }
 
 // ---- TMA tensor maps ----
@@ -96,12 +130,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// Pool [num_blocks][64][576] bf16 viewed as 3-D (col, token, page); box = 64 cols x 64 tokens.
-int make_kv_map(CUtensorMap* m, const void* kv, int num_blocks) {
+// Pool [num_blocks][64][row_width] bf16 viewed as 3-D (col, token, page); box = 64 cols x 64 tokens.
+int make_kv_map(CUtensorMap* m, const void* kv, int num_blocks, int row_width = kDqk) {
     auto enc = get_encode_fn();
     if (!enc) return MLA_ERR_CUDA;
-    cuuint64_t dims[3] = {(cuuint64_t)kDqk, (cuuint64_t)kPage, (cuuint64_t)num_blocks};
-    cuuint64_t strides[2] = {(cuuint64_t)kDqk * 2, (cuuint64_t)kDqk * 2 * kPage};
+    cuuint64_t dims[3] = {(cuuint64_t)row_width, (cuuint64_t)kPage, (cuuint64_t)num_blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)row_width * 2, (cuuint64_t)row_width * 2 * kPage};
     cuuint32_t box[3] = {64, (cuuint32_t)kPage, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box,
@@ -110,13 +144,13 @@ int make_kv_map(CUtensorMap* m, const void* kv, int num_blocks) {
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// Q [B*s_q*h][576] bf16 as 2-D; box = 64 cols x NG rows (rows past the end read as zero).
-int make_q_map(CUtensorMap* m, const void* q, int rows, int NG) {
+// Q [B*s_q*h][width] bf16 as 2-D; box = 64 cols x box_rows rows (rows past the end read as zero).
+int make_q_map(CUtensorMap* m, const void* q, int rows, int box_rows, int width = kDqk) {
     auto enc = get_encode_fn();
     if (!enc) return MLA_ERR_CUDA;
-    cuuint64_t dims[2] = {(cuuint64_t)kDqk, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kDqk * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)NG};
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -124,7 +158,7 @@ int make_q_map(CUtensorMap* m, const void* q, int rows, int NG) {
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-template <int NG>
+template <int NG, class S>
 int ensure_smem_attr() {
     static bool done[kMaxDevices] = {};
     static std::mutex mu;
@@ -132,16 +166,16 @@ int ensure_smem_attr() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
-        if (cudaFuncSetAttribute(mla_decode_fwd_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 FwdSmem<NG>::kAlloc) != cudaSuccess)
+        if (cudaFuncSetAttribute(mla_decode_fwd_kernel<NG, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FwdSmem<NG, S>::kAlloc) != cudaSuccess)
             return MLA_ERR_CUDA;
-        if constexpr (FwdWarps<NG>::kSplitRegs) {
+        if constexpr (FwdWarps<NG, S>::kSplitRegs) {
             // setmaxnreg.inc waits until the registers it asks for are free in
             // the CTA, so the split must fit the launch allocation exactly as
             // compiled; refuse to launch otherwise.
-            using Wp = FwdWarps<NG>;
+            using Wp = FwdWarps<NG, S>;
             cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, mla_decode_fwd_kernel<NG>) != cudaSuccess) return MLA_ERR_CUDA;
+            if (cudaFuncGetAttributes(&fa, mla_decode_fwd_kernel<NG, S>) != cudaSuccess) return MLA_ERR_CUDA;
             if ((long)fa.numRegs * Wp::kThreads < (long)Wp::kRegsIssue * 128 + (long)Wp::kRegsSoftmax * Wp::kSoftmaxThreads)
                 return MLA_ERR_UNSUPPORTED;
         }
@@ -150,48 +184,56 @@ int ensure_smem_attr() {
     return MLA_OK;
 }
 
-template <int NG>
+template <int NG, class S>
 int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const CUtensorMap& qm,
                cudaStream_t stream) {
-    int rc = ensure_smem_attr<NG>();
+    int rc = ensure_smem_attr<NG, S>();
     if (rc != MLA_OK) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.G);
-    cfg.blockDim = dim3(FwdWarps<NG>::kThreads);
-    cfg.dynamicSmemBytes = FwdSmem<NG>::kAlloc;
+    cfg.blockDim = dim3(FwdWarps<NG, S>::kThreads);
+    cfg.dynamicSmemBytes = FwdSmem<NG, S>::kAlloc;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mla_decode_fwd_kernel<NG>, kvm, qm, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, mla_decode_fwd_kernel<NG, S>, kvm, qm, p) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedule, const void* workspace,
-                   void* out, float* lse, cudaStream_t stream) {
+// Query-column layout of the work items, for the kernels' item_col().
+struct ColMap {
+    int s_q, heads, run_rows, run_stride;
+};
+
+template <int kDvT>
+int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const void* workspace, void* out,
+                   float* lse, cudaStream_t stream) {
     CombineParams c;
     c.sched = static_cast<const int32_t*>(schedule);
     c.opart = static_cast<const float*>(workspace);
-    c.lpart = c.opart + (size_t)pl.slots * pl.gr.NG * kDv;
+    c.lpart = c.opart + (size_t)pl.slots * pl.gr.NG * kDvT;
     c.out = static_cast<__nv_bfloat16*>(out);
     c.lse = lse;
     c.status = const_cast<int32_t*>(c.sched) + kHdrStatus;
-    c.s_q = d->s_q;
-    c.heads = d->num_heads;
+    c.s_q = cm.s_q;
+    c.heads = cm.heads;
     c.N = pl.gr.N;
     c.NG = pl.gr.NG;
     c.Hg = pl.gr.Hg;
     c.G = pl.G;
     c.BG = pl.BG;
     c.slots_cap = (int)pl.slots;
+    c.run_rows = cm.run_rows;
+    c.run_stride = cm.run_stride;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.BG, pl.gr.NG);
-    cfg.blockDim = dim3(kCombineThreads);
+    cfg.blockDim = dim3(kDvT / 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -199,12 +241,14 @@ int launch_combine(const mla_decode_dims* d, const Plan& pl, const void* schedul
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel, c) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel<kDvT>, c) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
+
+ColMap mla_colmap(const mla_decode_dims* d, const Plan& pl) { return ColMap{d->s_q, d->num_heads, pl.gr.NG, 0}; }
 
 // ---- scratch of the allocation-free entry point ----
 // One array per device, in this library's module; allocated by the driver when
@@ -363,12 +407,15 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = pl.gr.NG == 16   ? launch_fwd<16>(pl, p, kvm, qm, st)
-         : pl.gr.NG == 32 ? launch_fwd<32>(pl, p, kvm, qm, st)
-                          : launch_fwd<64>(pl, p, kvm, qm, st);
+    p.run_rows = pl.gr.NG;
+    p.run_stride = 0;
+    p.kv_groups = 1;
+    rc = pl.gr.NG == 16   ? launch_fwd<16, ShapeMla>(pl, p, kvm, qm, st)
+         : pl.gr.NG == 32 ? launch_fwd<32, ShapeMla>(pl, p, kvm, qm, st)
+                          : launch_fwd<64, ShapeMla>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
-    return launch_combine(dims, pl, schedule, workspace, out, lse, st);
+    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, st);
 }
 
 int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const void* workspace, void* out,
@@ -378,7 +425,93 @@ int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const 
     if (rc != MLA_OK) return rc;
     if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
-    return launch_combine(dims, pl, schedule, workspace, out, lse, static_cast<cudaStream_t>(stream));
+    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse,
+                               static_cast<cudaStream_t>(stream));
+}
+
+size_t mla_gqa_decode_schedule_bytes(const mla_gqa_dims* dims) {
+    Plan pl;
+    if (make_plan_gqa(dims, &pl) != MLA_OK) return 0;
+    return (size_t)schedule_words(pl.G, pl.BG) * sizeof(int32_t);
+}
+
+size_t mla_gqa_decode_workspace_bytes(const mla_gqa_dims* dims) {
+    Plan pl;
+    if (make_plan_gqa(dims, &pl) != MLA_OK) return 0;
+    return workspace_bytes_of(pl, ShapeGqa::kDv);
+}
+
+int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_seqlens, void* schedule,
+                                void* stream) {
+    Plan pl;
+    int rc = make_plan_gqa(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
+    const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
+    const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
+    mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
+        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.gr.Hg, pl.gr.NG, pl.G,
+        dims->max_blocks_per_seq, use_smem);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* workspace, const void* q,
+                       const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
+                       float softmax_scale, void* out, float* lse, void* stream) {
+    Plan pl;
+    int rc = make_plan_gqa(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(q) || !aligned16(kv_cache) ||
+        !aligned16(block_table) || !aligned16(cache_seqlens) || !aligned16(out) || !aligned16(lse))
+        return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    CUtensorMap kvm, qm;
+    rc = make_kv_map(&kvm, kv_cache, dims->num_blocks, ShapeGqa::row_width(dims->num_kv_groups));
+    if (rc != MLA_OK) return rc;
+    rc = make_q_map(&qm, q, dims->batch * pl.gr.N, kGqaHeadsPerGroup, ShapeGqa::kDqk);
+    if (rc != MLA_OK) return rc;
+    FwdParams p;
+    p.sched = static_cast<const int32_t*>(schedule);
+    p.block_table = block_table;
+    p.seqlens = cache_seqlens;
+    p.kv = static_cast<const uint8_t*>(kv_cache);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.opart = static_cast<float*>(workspace);
+    p.lpart = p.opart + (size_t)pl.slots * pl.gr.NG * ShapeGqa::kDv;
+    p.status = const_cast<int32_t*>(p.sched) + kHdrStatus;
+    p.s_q = dims->s_q;
+    p.heads = dims->num_q_heads;
+    p.N = pl.gr.N;
+    p.num_blocks = dims->num_blocks;
+    p.max_blocks = dims->max_blocks_per_seq;
+    p.causal = dims->causal;
+    p.G = pl.G;
+    p.BG = pl.BG;
+    p.Hg = pl.gr.Hg;
+    p.slots_cap = (int)pl.slots;
+    p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+    p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
+    p.run_rows = kGqaHeadsPerGroup;  // one run of 16 heads per new token
+    p.run_stride = dims->num_q_heads;
+    p.kv_groups = dims->num_kv_groups;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = pl.gr.NG == 16 ? launch_fwd<16, ShapeGqa>(pl, p, kvm, qm, st) : launch_fwd<32, ShapeGqa>(pl, p, kvm, qm, st);
+    if (rc != MLA_OK) return rc;
+    if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
+    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
+                                         pl, schedule, workspace, out, lse, st);
+}
+
+int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,
+                           float* lse, void* stream) {
+    Plan pl;
+    int rc = make_plan_gqa(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
+        return MLA_ERR_INVALID_ARG;
+    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
+                                         pl, schedule, workspace, out, lse, static_cast<cudaStream_t>(stream));
 }
 
 #ifdef MLA_TRACE

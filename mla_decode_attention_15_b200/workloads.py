@@ -176,3 +176,44 @@ def make_inputs(workload, seed: Optional[int] = None) -> dict:
               spare_pages=w.spare_pages, causal=w.causal)
     d["workload"] = w
     return d
+
+
+# ---------------------------------------------------------------- GQA path
+GQA_D_HEAD = 128
+GQA_D_ROPE = 64
+GQA_HEADS_PER_GROUP = 16
+
+
+def build_gqa(batch: int, s_q: int, groups: int, lens, sigma: float = 1.0, seed: int = 0,
+              spare_pages: int = 8, causal: bool = False, pool_device: str = "cpu") -> dict:
+    """Inputs for the GQLA GQA path: a group-expanded paged cache whose
+    per-token row is K_0..K_{g-1} (128 each), V_0..V_{g-1} (128 each), then the
+    shared RoPE key (64); 16 query heads per group, q = [B, s_q, 16g, 192].
+    Draw order as in build(): lengths, Q, pool (on ``pool_device``), block
+    table permutation.  No attention arithmetic here."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    seqlens = _draw_lens(lens, batch, g)
+    pages = [(int(L) + PAGE - 1) // PAGE for L in seqlens.tolist()]
+    max_pages = max(max(pages) if pages else 0, 1)
+    h = GQA_HEADS_PER_GROUP * groups
+    width = 2 * groups * GQA_D_HEAD + GQA_D_ROPE
+    q = (torch.randn(batch * s_q * h * (GQA_D_HEAD + GQA_D_ROPE), generator=g) * sigma).to(torch.bfloat16)
+    q = q.view(batch, s_q, h, GQA_D_HEAD + GQA_D_ROPE)
+    num_blocks = sum(pages) + spare_pages
+    n = num_blocks * PAGE * width
+    if pool_device == "cpu":
+        kv = (torch.randn(n, generator=g) * sigma).to(torch.bfloat16)
+    else:
+        gd = torch.Generator(device=pool_device)
+        gd.manual_seed(int(seed) + 1)
+        kv = (torch.randn(n, generator=gd, device=pool_device) * sigma).to(torch.bfloat16)
+    kv = kv.view(num_blocks, PAGE, 1, width)
+    ids = torch.randperm(num_blocks, generator=g).to(torch.int32)
+    block_table = torch.full((batch, max_pages), -1, dtype=torch.int32)
+    k = 0
+    for b, P in enumerate(pages):
+        block_table[b, :P] = ids[k:k + P]
+        k += P
+    return dict(q=q, kv_cache=kv, block_table=block_table, cache_seqlens=seqlens,
+                softmax_scale=SOFTMAX_SCALE, causal=bool(causal), groups=groups)
