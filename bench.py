@@ -51,6 +51,9 @@ def parse_args():
                     help="decode only the first BATCH requests of the workload (small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--gqa", action="store_true",
+                    help="GQA path over a group-expanded cache (bs16, s_q 2 causal, 8 KV groups = 128 query "
+                         "heads, 16K context): one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="context/batch sweep (bs x L grid, 16 heads, s_q 1): one JSON line per point "
                          "instead of the single bench line")
@@ -610,10 +613,84 @@ def run_sweep(args):
     return 0
 
 
+def run_gqa_bench(args):
+    """The GQLA GQA path (group-expanded cache: per token 8 groups of 128-wide
+    keys and values plus a 64-wide shared RoPE key) at bs16, s_q 2 causal,
+    128 query heads, 16K context: step (schedule + decode + combine) and
+    decode kernel alone, graph-replayed; bytes = every cache row once + Q + O
+    + LSE, FLOPs = 2 * h_q * s_q * L * (192 + 128)."""
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    bd.lib()
+    stream = torch.cuda.current_stream(dev)
+    B, s_q, groups, L = 16, 2, 8, 16384
+    h = 16 * groups
+    d = workloads.build_gqa(B, s_q, groups, ("fixed", L), seed=1005, causal=True, pool_device="cuda")
+    q, kv = d["q"].to(dev), d["kv_cache"]
+    bt, sl = d["block_table"].to(dev), d["cache_seqlens"].to(dev)
+    dims = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0)
+    dnc = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0, bd.MLA_FLAG_NO_COMBINE)
+    sched = torch.empty(bd.mla_gqa_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
+    ws = torch.empty(bd.mla_gqa_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, s_q, h, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, h, s_q, dtype=torch.float32, device=dev)
+    tokens = kv_tokens(d["cache_seqlens"])
+    kv_bytes = tokens * (2 * groups * 128 + 64) * 2
+    total_bytes = kv_bytes + q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
+    flops = 2 * h * s_q * tokens * (192 + 128)
+
+    def step(st, dm):
+        bd.mla_gqa_decode_get_schedule(dm, sl, sched, st)
+        bd.mla_gqa_decode_fwd(dm, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
+
+    times = []
+    for dm in (dims, dnc):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            step(cap, dm)
+            with torch.cuda.graph(g, stream=cap):
+                step(cap, dm)
+        stream.wait_stream(cap)
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) / args.steps)
+        del g
+    status = bd.mla_decode_get_status(sched)
+    assert status == 0, "device status %#x" % status
+    ms_step, ms_kernel = times
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    line = {
+        "metric": "GQA-path decode (group-expanded cache) KV GB/s", "value": kv_bytes / (ms_step * 1e-3) / 1e9,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "us_per_call": ms_step * 1e3, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "impl": "ours",
+        "config": {"workload": "gqa_b16_sq2_g8_l16k: batch 16, s_q 2 causal, 8 KV groups x 16 query heads, "
+                               "KV len 16384, d_head 128 + shared RoPE 64, permuted pages",
+                   "kv_bytes_per_step": kv_bytes, "l2": "inputs larger than L2 (1.1 GB): no flush"},
+        "kernel_us": ms_kernel * 1e3, "tflops": flops / (ms_step * 1e-3) / 1e12,
+        "roofline": kernel_roofline({"total": total_bytes}, flops, ms_kernel, hbm_peak, tf_peak, peak_kind, None),
+        "gpu_launches": 3 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.sweep:
         return run_sweep(args)
+    if args.gqa:
+        return run_gqa_bench(args)
     w = workloads.WORKLOADS[args.workload]
     if args.batch:
         import dataclasses

@@ -71,6 +71,7 @@ struct ShapeMla {
     static constexpr int kRopeBox = 8;
     static constexpr int kVChunks = 4;     // d_v / 128: GEMM2 chunks of 128 rows
     static constexpr bool kPrefetchL2 = true;  // a page is one contiguous 72 KB block
+    static constexpr int kStages = 2;          // 72 KB page stages
     __host__ __device__ static constexpr int k_box(int c) { return c; }
     // first stage box of d_v chunk ch; the chunk's second box follows 8 KB on
     __host__ __device__ static constexpr int v_box(int ch) { return 2 * ch; }
@@ -86,6 +87,7 @@ struct ShapeGqa {
     static constexpr int kRopeBox = 2;
     static constexpr int kVChunks = 1;
     static constexpr bool kPrefetchL2 = false;  // a group's boxes are strided across the page
+    static constexpr int kStages = 4;           // 40 KB page stages
     __host__ __device__ static constexpr int k_box(int c) { return c; }
     __host__ __device__ static constexpr int v_box(int) { return 3; }
     __host__ __device__ static constexpr int col(int c, int kg, int kv_groups) {
@@ -229,9 +231,10 @@ struct CombineParams {
 };
 
 // ------------------------------------------------------------------ layout
+constexpr int kMaxStages = 4;
 template <int NG, class S = ShapeMla>
 struct FwdSmem {
-    static constexpr int kStages = 2;
+    static constexpr int kStages = S::kStages;
     static constexpr int kBoxCols = 64;
     static constexpr int kBoxBytes = kPage * kBoxCols * 2;    // 8 KB: 64 tokens x 64 cols
     static constexpr int kBoxes = S::kStageBoxes;             // boxes per page (9 for MLA)
@@ -258,7 +261,7 @@ struct FwdSmem {
     static constexpr int kSumQOff = kRedOff + 2 * NG * 4 * 4;  // float [NG][4]: sums of the bf16 P
     static constexpr int kVoteOff = kSumQOff + NG * 4 * 4;     // uint32 [2][8]: per-warp growth votes
     static constexpr int kBarOff = kVoteOff + 2 * 8 * 4;
-    static constexpr int kNumBars = 24;
+    static constexpr int kNumBars = 32;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMiscOff + 16;
     // Slack to align the base to 1 KB where it fits; without it the kernel
@@ -276,12 +279,16 @@ struct FwdSmem {
     static_assert(kQOff % 1024 == 0 && kStageBytes % 1024 == 0 && kPInStage % 1024 == 0,
                   "swizzle atoms need 1 KB alignment");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kStages >= 2 && kStages <= kMaxStages, "stage count");
 };
 
 enum Bar {
-    kKvFull0 = 0, kKvFull1, kKvEmpty0, kKvEmpty1, kQFull, kQEmpty,
+    kQFull = 0, kQEmpty,
     kSFull0, kSFull1, kSEmpty0, kSEmpty1, kPFull0, kPFull1, kPEmpty0, kPEmpty1,
-    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kMaxFull, kBarCount
+    kOEmpty, kMmaDone, kRedFull0, kRedFull1, kSumFull, kMmaDone2, kOutStaged, kOutFree, kMaxFull,
+    kKvFull0,                             // kMaxStages "page landed" barriers
+    kKvEmpty0 = kKvFull0 + kMaxStages,    // kMaxStages "stage free" barriers
+    kBarCount = kKvEmpty0 + kMaxStages
 };
 static_assert(kBarCount <= FwdSmem<16>::kNumBars, "barrier slots");
 
@@ -483,7 +490,7 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     it.init(meta);
     Item item;
     uint32_t kv_it = 0, q_it = 0;
-    uint32_t issued0 = 0, issued1 = 0;  // pages loaded per stage (for the abort drain)
+    uint32_t issued[kMaxStages] = {};  // pages loaded per stage (for the abort drain)
     bool stall = p.test_stall != 0;
     bool ok = true;
     MLA_TRACE_DECL(0);
@@ -515,8 +522,8 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
                 if ((unsigned)ph < (unsigned)p.num_blocks)
                     prefetch_l2_bulk(p.kv + (size_t)ph * L::kStageBytes, L::kStageBytes);
             }
-            const int st = kv_it & 1;
-            ok = wait_bounded(bar0 + 8 * (kKvEmpty0 + st), ((kv_it >> 1) & 1) ^ 1, ctl);
+            const int st = kv_it % L::kStages;
+            ok = wait_bounded(bar0 + 8 * (kKvEmpty0 + st), ((kv_it / L::kStages) & 1) ^ 1, ctl);
             if (!ok) break;
             if (stall) {  // test hook: this page is never loaded, so its GEMM1 wait runs out
                 stall = false;
@@ -536,15 +543,16 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
             for (int c = 0; c < L::kBoxes; ++c)
                 tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, S::col(c, item.g, p.kv_groups), 0, phys,
                                  policy);
-            issued0 += st == 0;
-            issued1 += st == 1;
+#pragma unroll
+            for (int k = 0; k < L::kStages; ++k) issued[k] += st == k;
             ++kv_it;
         }
     }
     if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        if (issued0 > 0) wait_drain(bar0 + 8 * kKvFull0, (issued0 - 1) & 1);
-        if (issued1 > 0) wait_drain(bar0 + 8 * kKvFull1, (issued1 - 1) & 1);
+#pragma unroll
+        for (int k = 0; k < L::kStages; ++k)
+            if (issued[k] > 0) wait_drain(bar0 + 8 * (kKvFull0 + k), (issued[k] - 1) & 1);
         if (q_it > 0) wait_drain(bar0 + 8 * kQFull, (q_it - 1) & 1);
     }
 }
@@ -578,16 +586,16 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
         ok = wait_bounded(bar0 + 8 * kQFull, q_it & 1, ctl);
         if (!ok) break;
         for (int j = item.p0; j < item.p1; ++j) {
-            const int st = s_it & 1;
-            const uint32_t par = (s_it >> 1) & 1;
-            ok = wait_bounded(bar0 + 8 * (kKvFull0 + st), par, ctl);
+            const int st = s_it % L::kStages;  // KV stage of the page
+            const int sb = s_it & 1;            // S^T buffer
+            ok = wait_bounded(bar0 + 8 * (kKvFull0 + st), (s_it / L::kStages) & 1, ctl);
             if (!ok) break;
             MLA_TRACE_EV(kTrMmaKvFull);
-            ok = wait_bounded(bar0 + 8 * (kSEmpty0 + st), par ^ 1, ctl);
+            ok = wait_bounded(bar0 + 8 * (kSEmpty0 + sb), ((s_it >> 1) & 1) ^ 1, ctl);
             if (!ok) break;
             tc_fence_after();
             // This issuer's accumulator; it takes boxes issuer, issuer + 2, ...
-            const uint32_t d = tmem + L::kSCol + (st * G1<NG>::kIssuers + issuer) * NG;
+            const uint32_t d = tmem + L::kSCol + (sb * G1<NG>::kIssuers + issuer) * NG;
             const uint64_t a_st = a_desc0 + ((st * L::kStageBytes) >> 4);
             bool first = true;
 #pragma unroll 1
@@ -601,7 +609,7 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
                 }
             }
             issued = true;
-            umma_commit(bar0 + 8 * (kSFull0 + st));
+            umma_commit(bar0 + 8 * (kSFull0 + sb));
             MLA_TRACE_EV(kTrMmaG1Issued);
             if (j == item.p1 - 1) umma_commit(bar0 + 8 * kQEmpty);
             ++s_it;
@@ -642,9 +650,10 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NG * 2, kPSwizzle);
     while (ok && it.next(p, bginfo, item)) {
         for (int j = item.p0; j < item.p1; ++j) {
-            const int st = s_it & 1;
+            const int st = s_it % L::kStages;  // KV stage of the page (holds its P^T)
+            const int pb = s_it & 1;            // P^T handoff barriers
             const bool first = (j == item.p0);
-            ok = wait_bounded(bar0 + 8 * (kPFull0 + st), (s_it >> 1) & 1, ctl);
+            ok = wait_bounded(bar0 + 8 * (kPFull0 + pb), (s_it >> 1) & 1, ctl);
             if (!ok) break;
             if (first) {
                 ok = wait_bounded(bar0 + 8 * kOEmpty, (item_it & 1) ^ 1, ctl);
@@ -666,7 +675,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             }
             issued = true;
             umma_commit(bar0 + 8 * (kKvEmpty0 + st));
-            umma_commit(bar0 + 8 * (kPEmpty0 + st));
+            umma_commit(bar0 + 8 * (kPEmpty0 + pb));
             MLA_TRACE_EV(kTrMmaG2Issued);
             ++s_it;
         }
@@ -812,8 +821,8 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             float e[W];
 #pragma unroll
             for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
-            const int pb = s_it & 1;                      // the page's stage
-            uint8_t* rowp = pbuf + pb * L::kStageBytes + row * (NG * 2);
+            const int pb = s_it & 1;                      // P^T handoff barriers
+            uint8_t* rowp = pbuf + (s_it % L::kStages) * L::kStageBytes + row * (NG * 2);  // the page's stage
             auto store_p = [&](const float (&ev)[W]) {
                 uint32_t packed[W / 2];
 #pragma unroll
@@ -1134,7 +1143,8 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
                 i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged || i == kMaxFull)
                 count = FwdWarps<NG, S>::kSoftmaxThreads;
             if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
-            if (i == kKvEmpty0 || i == kKvEmpty1 || i == kPEmpty0 || i == kPEmpty1 || i == kMmaDone2)
+            if ((i >= kKvEmpty0 && i < kKvEmpty0 + kMaxStages) || i == kPEmpty0 || i == kPEmpty1 ||
+                i == kMmaDone2)
                 count = FwdWarps<NG, S>::kG2Issuers;
             mbar_init(bar0 + 8 * i, count);
         }
