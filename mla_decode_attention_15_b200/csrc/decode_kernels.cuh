@@ -113,7 +113,9 @@ struct FwdWarps {
     static constexpr int kG2Issuers = NG == 16 && S::kVChunks >= 4 ? 4 : 1;  // 4: one per d_v chunk
     static constexpr int kFirstG2 = 1 + G1<NG>::kIssuers;
     static constexpr int kFirstSoftmax = kFirstG2 + kG2Issuers;
-    static constexpr int kColGroups = NG == 64 ? 2 : 1;   // softmax column groups
+    // softmax column groups: 64-column MLA groups, and 32-column GQA groups
+    // (whose 40 KB pages leave the softmax as the serial step)
+    static constexpr int kColGroups = NG == 64 || (NG == 32 && S::kVChunks == 1) ? 2 : 1;
     static constexpr int kGroupCols = NG / kColGroups;     // query columns per group
     static constexpr int kSoftmaxThreads = 128 * kColGroups;
     static constexpr int kThreads = 32 * kFirstSoftmax + kSoftmaxThreads;
@@ -252,7 +254,9 @@ struct FwdSmem {
     static constexpr int kQOff = kKvOff + kStages * kStageBytes;
     // 64-column groups: Q^T takes 72 KB, so the epilogue stores straight from
     // registers (no staging tile).
-    static constexpr int kOutRows = NG == 64 ? 0 : 16;        // output rows (query columns) per staging pass
+    // output rows (query columns) per staging pass; column-grouped softmax
+    // warps store from registers instead
+    static constexpr int kOutRows = FwdWarps<NG, S>::kColGroups > 1 ? 0 : 16;
     static constexpr int kOutOff = kQOff + kQBytes;           // staging: [16][d_v] fp32 (or bf16)
     static constexpr int kOutBytes = kOutRows * S::kDv * 4;
     // float [2][NG][4]: page maxima of the 4 lane quadrants, double-buffered
