@@ -128,3 +128,11 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_build, "LIB", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         bd.lib()
+
+
+def test_build_entry_point_compiles_and_imports():
+    """The build check: __graft_entry__.build() compiles (or finds up to date)
+    the library and the oracle and imports the package at the ABI version it
+    expects."""
+    import __graft_entry__
+    __graft_entry__.build()
