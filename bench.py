@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--gqa", action="store_true",
                     help="GQA path over a group-expanded cache (bs16, s_q 2 causal, 8 KV groups = 128 query "
                          "heads, 16K context): one JSON line")
+    ap.add_argument("--absorb", action="store_true",
+                    help="absorbed projections q_nope.W_UK and O.W_UV at decode sizes (bs16 x 16 heads, "
+                         "bs32 x s_q 2 x 128 heads): one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="context/batch sweep (bs x L grid, 16 heads, s_q 1): one JSON line per point "
                          "instead of the single bench line")
@@ -685,8 +688,90 @@ def run_gqa_bench(args):
     return 0
 
 
+def run_absorb_bench(args):
+    """The absorbed projections around the decode (GQLA summary, "Caminho
+    MQA-Absorvido") at the decode batches of the two measured configurations.
+    Each case holds the weights of 61 layers and calls layer i for call i, the
+    way one decode step runs through a model, so the weights (4 or 32 MB per
+    layer) come from HBM, not L2.  Graph-replayed; per-call time = replay time
+    / 61.  Algorithmic bytes: weights + input rows + output rows, once."""
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    bd.lib()
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, _, peak_kind = measured_peaks()
+    layers = 61
+    cases = []
+    for name, T, h in (("b16_sq1_h16", 16, 16), ("b32_sq2_h128", 64, 128)):
+        x = workloads.build_absorb(T, h, seed=1200 + h)
+        q_in, o = x["q_in"].to(dev), x["o"].to(dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(1300 + h)
+        w_uk = (torch.randn(layers, h, 128, 512, generator=g, device=dev) / 128 ** 0.5).to(torch.bfloat16)
+        w_uv = (torch.randn(layers, h, 512, 128, generator=g, device=dev) / 512 ** 0.5).to(torch.bfloat16)
+        q_out = torch.empty(T, h, 576, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(T, h, 128, dtype=torch.bfloat16, device=dev)
+        status = torch.zeros(4, dtype=torch.int32, device=dev)
+        dims = bd.make_absorb_dims(T, h)
+        res = {}
+        for kind in ("absorb_q", "absorb_o"):
+            def calls(st, kind=kind):
+                for i in range(layers):
+                    if kind == "absorb_q":
+                        bd.mla_absorb_q(dims, q_in, w_uk[i], q_out, status, st)
+                    else:
+                        bd.mla_absorb_o(dims, o, w_uv[i], out, status, st)
+            graph = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream()
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                calls(cap)
+                with torch.cuda.graph(graph, stream=cap):
+                    calls(cap)
+            stream.wait_stream(cap)
+            for _ in range(max(3, args.warmup)):
+                graph.replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / (args.steps * layers)
+            del graph
+            w_bytes = h * 128 * 512 * 2
+            io = T * h * (192 + 576) * 2 if kind == "absorb_q" else T * h * (512 + 128) * 2
+            byt = w_bytes + io
+            achieved = byt / (us * 1e-6) / 1e9
+            res[kind] = {"us_per_call": us, "algorithmic_bytes": byt, "achieved_gbs": achieved,
+                         "frac": achieved / hbm_peak, "tflops": 2 * T * h * 128 * 512 / (us * 1e-6) / 1e12}
+        assert int(status.max()) == 0, "device status %#x" % int(status.max())
+        cases.append({"case": name, "tokens": T, "heads": h, **res})
+    main_case = cases[1]
+    us = main_case["absorb_q"]["us_per_call"] + main_case["absorb_o"]["us_per_call"]
+    byt = main_case["absorb_q"]["algorithmic_bytes"] + main_case["absorb_o"]["algorithmic_bytes"]
+    line = {
+        "metric": "absorbed projections (q_nope.W_UK + O.W_UV) GB/s", "value": byt / (us * 1e-6) / 1e9,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": us * 1e-3,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": {"workload": "absorb_b32_sq2_h128: 64 tokens x 128 heads, W_UK [128,128,512] + "
+                               "W_UV [128,512,128] per layer, 61 layers in rotation",
+                   "l2": "61 layers of weights (244 MB / 2 GB) rotate: no flush"},
+        "roofline": {"kernel": "mla_absorb_kernel", "bound": "hbm", "achieved": byt / (us * 1e-6) / 1e9,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": byt / (us * 1e-6) / 1e9 / hbm_peak,
+                     "peak_kind": peak_kind + " (copy bandwidth, burst)", "traffic": None},
+        "cases": cases, "gpu_launches": 2 * layers * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.absorb:
+        return run_absorb_bench(args)
     if args.sweep:
         return run_sweep(args)
     if args.gqa:

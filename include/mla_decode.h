@@ -231,6 +231,48 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
 int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,
                            float* lse, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Absorbed projections around the decode (GQLA technical summary,
+ * gist.science, pt, 2605.15250, "Caminho MQA-Absorvido": the key and value
+ * up-projections are absorbed into the query and output projections, so every
+ * head attends to the 512-wide latent cache directly).  Per token t and head h:
+ *
+ *   mla_absorb_q:  q_out[t][h] = [ q_in[t][h][0:128] . w_uk[h]  |  q_in[t][h][128:192] ]
+ *                  (512-wide latent query, then the 64-wide RoPE part unchanged:
+ *                  exactly the q layout mla_decode_fwd takes)
+ *   mla_absorb_o:  out[t][h]   =   o[t][h][0:512] . w_uv[h]
+ *                  (the decode output over latent rows to the head's 128-wide
+ *                  value space)
+ *
+ *   q_in   bf16 [tokens][num_heads][192]      w_uk  bf16 [num_heads][128][512]
+ *   q_out  bf16 [tokens][num_heads][576]
+ *   o      bf16 [tokens][num_heads][512]      w_uv  bf16 [num_heads][512][128]
+ *   out    bf16 [tokens][num_heads][128]
+ * All row-major and contiguous; tokens = batch * s_q.  Products accumulate in
+ * fp32 and round once to bf16.  Every pointer is device memory owned by the
+ * caller, 16-byte aligned; input and output must not overlap.  status is an
+ * optional device int32 (NULL or 4-byte aligned) into which a kernel ORs
+ * MLA_STATUS_TIMEOUT if one of its waits gave up (after ~1 s; the output is
+ * then incomplete).  Work is enqueued on `stream` (NULL = legacy default);
+ * nothing is allocated.  Returns MLA_ERR_INVALID_ARG for a NULL or
+ * misaligned pointer, tokens outside [1, 4194240] or num_heads outside
+ * [1, 65535]; MLA_ERR_UNSUPPORTED unless d_nope 128, d_rope 64, d_latent 512,
+ * d_v_head 128; MLA_ERR_CUDA if a launch fails.
+ * ---------------------------------------------------------------------- */
+typedef struct mla_absorb_dims {
+    int32_t tokens;    /* T >= 1 */
+    int32_t num_heads; /* h >= 1 */
+    int32_t d_nope;    /* must be 128 */
+    int32_t d_rope;    /* must be 64 */
+    int32_t d_latent;  /* must be 512 */
+    int32_t d_v_head;  /* must be 128 */
+} mla_absorb_dims;
+
+int mla_absorb_q(const mla_absorb_dims* dims, const void* q_in, const void* w_uk, void* q_out,
+                 int32_t* status, void* stream);
+int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, void* out,
+                 int32_t* status, void* stream);
+
 /* Library ABI version (increments on any change of these declarations). */
 int mla_decode_version(void);
 

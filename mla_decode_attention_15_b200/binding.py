@@ -52,11 +52,18 @@ EXPORTED = (
     "mla_gqa_decode_get_schedule",
     "mla_gqa_decode_fwd",
     "mla_gqa_decode_combine",
+    "mla_absorb_q",
+    "mla_absorb_o",
 )
 
 GQA_D_HEAD = 128
 GQA_D_ROPE = 64
 GQA_HEADS_PER_GROUP = 16
+
+ABSORB_D_NOPE = 128
+ABSORB_D_ROPE = 64
+ABSORB_D_LATENT = 512
+ABSORB_D_V_HEAD = 128
 
 
 class MlaDecodeError(RuntimeError):
@@ -75,6 +82,11 @@ class mla_gqa_dims(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "batch", "s_q", "num_q_heads", "num_kv_groups", "num_blocks", "max_blocks_per_seq", "page_size",
         "d_head", "d_rope", "causal", "num_sms", "flags")]
+
+
+class mla_absorb_dims(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "tokens", "num_heads", "d_nope", "d_rope", "d_latent", "d_v_head")]
 
 
 _lib = None
@@ -125,6 +137,10 @@ def lib() -> ctypes.CDLL:
         L.mla_gqa_decode_fwd.argtypes = [Q, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
         L.mla_gqa_decode_combine.restype = ctypes.c_int
         L.mla_gqa_decode_combine.argtypes = [Q, vp, vp, vp, vp, vp]
+        A = ctypes.POINTER(mla_absorb_dims)
+        for name in ("mla_absorb_q", "mla_absorb_o"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = [A, vp, vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -369,3 +385,60 @@ class GqaDecoder:
 
     def status(self) -> int:
         return mla_decode_get_status(self.schedule)
+
+
+# ---------------------------------------------------------------- absorbed projections
+def make_absorb_dims(tokens: int, num_heads: int) -> mla_absorb_dims:
+    return mla_absorb_dims(int(tokens), int(num_heads), ABSORB_D_NOPE, ABSORB_D_ROPE, ABSORB_D_LATENT,
+                           ABSORB_D_V_HEAD)
+
+
+def mla_absorb_q(dims: mla_absorb_dims, q_in, w_uk, q_out, status=None, stream=None) -> None:
+    _check(lib().mla_absorb_q(ctypes.byref(dims), _ptr(q_in), _ptr(w_uk), _ptr(q_out), _ptr(status),
+                              _stream(stream)), "mla_absorb_q")
+
+
+def mla_absorb_o(dims: mla_absorb_dims, o, w_uv, out, status=None, stream=None) -> None:
+    _check(lib().mla_absorb_o(ctypes.byref(dims), _ptr(o), _ptr(w_uv), _ptr(out), _ptr(status),
+                              _stream(stream)), "mla_absorb_o")
+
+
+def _bf16_on(t, shape, what, device):
+    _require(t.dtype == torch.bfloat16 and t.is_contiguous() and tuple(t.shape) == tuple(shape),
+             "%s must be contiguous bf16 %s" % (what, list(shape)))
+    _require(t.device == device, "%s must be on %s" % (what, device))
+
+
+def absorb_q(q_in: torch.Tensor, w_uk: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """q_in [..., h, 192] (each head's 128-wide part, then its RoPE part) and
+    w_uk [h, 128, 512] -> [..., h, 576]: the latent query q_nope . W_UK with the
+    RoPE part after it, the layout mla_decode takes as q."""
+    h = q_in.shape[-2]
+    T = q_in.numel() // (h * (ABSORB_D_NOPE + ABSORB_D_ROPE)) if q_in.numel() else 0
+    _require(T >= 1 and q_in.shape[-1] == ABSORB_D_NOPE + ABSORB_D_ROPE, "q_in must be [..., h, 192]")
+    _bf16_on(q_in, q_in.shape, "q_in", q_in.device)
+    _bf16_on(w_uk, (h, ABSORB_D_NOPE, ABSORB_D_LATENT), "w_uk", q_in.device)
+    shape = tuple(q_in.shape[:-1]) + (ABSORB_D_LATENT + ABSORB_D_ROPE,)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=q_in.device)
+    _bf16_on(out, shape, "out", q_in.device)
+    mla_absorb_q(make_absorb_dims(T, h), q_in, w_uk, out, None, stream)
+    return out
+
+
+def absorb_o(o: torch.Tensor, w_uv: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """o [..., h, 512] (the decode's output over latent rows) and w_uv
+    [h, 512, 128] -> [..., h, 128] = O . W_UV per head."""
+    h = o.shape[-2]
+    T = o.numel() // (h * ABSORB_D_LATENT) if o.numel() else 0
+    _require(T >= 1 and o.shape[-1] == ABSORB_D_LATENT, "o must be [..., h, 512]")
+    _bf16_on(o, o.shape, "o", o.device)
+    _bf16_on(w_uv, (h, ABSORB_D_LATENT, ABSORB_D_V_HEAD), "w_uv", o.device)
+    shape = tuple(o.shape[:-1]) + (ABSORB_D_V_HEAD,)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=o.device)
+    _bf16_on(out, shape, "out", o.device)
+    mla_absorb_o(make_absorb_dims(T, h), o, w_uv, out, None, stream)
+    return out

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "absorb_kernels.cuh"
 #include "decode_kernels.cuh"
 #include "mla_decode.h"
 #include "schedule.cuh"
@@ -17,7 +18,7 @@ namespace {
 
 using namespace mla;
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
 
 int validate_dims(const mla_decode_dims* d) {
@@ -278,6 +279,79 @@ int noalloc_scratch(void** out) {
     }
     *out = addr[dev];
     return MLA_OK;
+}
+
+// ---- absorbed projections ----
+int validate_absorb(const mla_absorb_dims* d) {
+    if (d == nullptr) return MLA_ERR_INVALID_ARG;
+    if (d->tokens < 1 || d->tokens > 65535 * kProjTokens || d->num_heads < 1 || d->num_heads > 65535)
+        return MLA_ERR_INVALID_ARG;
+    if (d->d_nope != kProjNope || d->d_rope != kProjRope || d->d_latent != kProjLatent ||
+        d->d_v_head != kProjVHead)
+        return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+// Per-head weight [h][rows][cols] bf16 as 3-D (col, row, head); box = 64 cols x box_rows rows.
+int make_weight_map(CUtensorMap* m, const void* w, int heads, int rows, int cols, int box_rows) {
+    auto enc = get_encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)heads};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * rows};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Token rows [T][h][width] bf16 as 3-D (col, head, token); box = 64 cols x 1 head x 64 tokens.
+int make_rows_map(CUtensorMap* m, const void* x, int T, int heads, int width) {
+    auto enc = get_encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)heads, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * 2 * heads};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kProjTokens};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <int kKind>
+int launch_absorb(const mla_absorb_dims* d, const void* x, const void* w, void* out, int32_t* status,
+                  cudaStream_t stream) {
+    using P = ProjShape<kKind>;
+    static bool done[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            if (cudaFuncSetAttribute(mla_absorb_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     P::kSmem) != cudaSuccess)
+                return MLA_ERR_CUDA;
+            done[dev] = true;
+        }
+    }
+    CUtensorMap wm, xm;
+    int rc = kKind == 0 ? make_weight_map(&wm, w, d->num_heads, kProjNope, kProjLatent, P::kWBoxRows)
+                        : make_weight_map(&wm, w, d->num_heads, kProjLatent, kProjVHead, P::kWBoxRows);
+    if (rc != MLA_OK) return rc;
+    rc = make_rows_map(&xm, x, d->tokens, d->num_heads, P::kInW);
+    if (rc != MLA_OK) return rc;
+    ProjParams p;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.rope_in = static_cast<const __nv_bfloat16*>(x);
+    p.status = status;
+    p.T = d->tokens;
+    p.heads = d->num_heads;
+    const dim3 grid(P::kChunks, d->num_heads, (d->tokens + kProjTokens - 1) / kProjTokens);
+    mla_absorb_kernel<kKind><<<grid, kProjThreads, P::kSmem, stream>>>(wm, xm, p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace
@@ -560,6 +634,24 @@ int mla_decode_get_status(const void* schedule, int32_t* host_status) {
         return MLA_ERR_CUDA;
     }
     return MLA_OK;
+}
+
+int mla_absorb_q(const mla_absorb_dims* dims, const void* q_in, const void* w_uk, void* q_out, int32_t* status,
+                 void* stream) {
+    int rc = validate_absorb(dims);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(q_in) || !aligned16(w_uk) || !aligned16(q_out)) return MLA_ERR_INVALID_ARG;
+    if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return MLA_ERR_INVALID_ARG;
+    return launch_absorb<0>(dims, q_in, w_uk, q_out, status, static_cast<cudaStream_t>(stream));
+}
+
+int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, void* out, int32_t* status,
+                 void* stream) {
+    int rc = validate_absorb(dims);
+    if (rc != MLA_OK) return rc;
+    if (!aligned16(o) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+    if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return MLA_ERR_INVALID_ARG;
+    return launch_absorb<1>(dims, o, w_uv, out, status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

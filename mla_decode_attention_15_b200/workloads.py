@@ -217,3 +217,26 @@ def build_gqa(batch: int, s_q: int, groups: int, lens, sigma: float = 1.0, seed:
         k += P
     return dict(q=q, kv_cache=kv, block_table=block_table, cache_seqlens=seqlens,
                 softmax_scale=SOFTMAX_SCALE, causal=bool(causal), groups=groups)
+
+
+ABSORB_D_NOPE, ABSORB_D_ROPE, ABSORB_D_LATENT, ABSORB_D_V_HEAD = 128, 64, 512, 128
+
+
+def build_absorb(tokens: int, heads: int, seed: int = 0, sigma: float = 1.0) -> dict:
+    """Inputs for the absorbed projections (GQLA summary, "Caminho
+    MQA-Absorvido"), all bf16 on the CPU, drawn in this order from one CPU
+    generator: q_in [T, h, 192] = randn * sigma; w_uk [h, 128, 512] = randn /
+    sqrt(128); o [T, h, 512] = randn * sigma; w_uv [h, 512, 128] = randn /
+    sqrt(512).  The weight scales keep the products near unit variance, as a
+    trained projection's would be; the weights themselves are random."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+
+    def draw(shape, scale):
+        return (torch.randn(math.prod(shape), generator=g) * scale).to(torch.bfloat16).view(*shape)
+
+    q_in = draw((tokens, heads, ABSORB_D_NOPE + ABSORB_D_ROPE), sigma)
+    w_uk = draw((heads, ABSORB_D_NOPE, ABSORB_D_LATENT), 1.0 / math.sqrt(ABSORB_D_NOPE))
+    o = draw((tokens, heads, ABSORB_D_LATENT), sigma)
+    w_uv = draw((heads, ABSORB_D_LATENT, ABSORB_D_V_HEAD), 1.0 / math.sqrt(ABSORB_D_LATENT))
+    return dict(q_in=q_in, w_uk=w_uk, o=o, w_uv=w_uv)

@@ -24,7 +24,7 @@ LSE_REL = 1e-5
 
 def header_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(mla_(?:gqa_)?decode_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(mla_(?:(?:gqa_)?decode|absorb)_\w+)\s*\(", text, re.M)))
 
 
 def bf16_floor(ref: np.ndarray) -> float:
