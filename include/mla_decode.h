@@ -273,6 +273,39 @@ int mla_absorb_q(const mla_absorb_dims* dims, const void* q_in, const void* w_uk
 int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, void* out,
                  int32_t* status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Split-KV across GPUs: merge of per-rank decode results.  Each of R ranks
+ * decodes the same queries against a disjoint part of every request's KV
+ * (for example a contiguous range of its pages, held in that rank's own
+ * pool); the ranks exchange their bf16 outputs and fp32 LSEs (an all-gather
+ * over NVLink) and each merges them with this call:
+ *
+ *   L* = log sum_i exp(lse_i),  out = sum_i exp(lse_i - L*) o_i,  lse = L*
+ *
+ * (the same LSE-weighted merge mla_decode_combine applies to the split
+ * partials inside one GPU).  A rank whose part is empty or fully masked
+ * reports lse_i = -inf and weighs nothing; a row with every lse_i = -inf gets
+ * out = 0 and lse = -inf.  For causal decode (s_q > 1), the rank that holds a
+ * request's last tokens runs with causal = 1 and every other rank with
+ * causal = 0: the causal rule only ever masks the request's last s_q - 1
+ * positions.
+ *
+ *   o_parts    bf16 [num_ranks][batch][s_q][num_heads][d_v]  (rank-major
+ *              stack of mla_decode_fwd / mla_gqa_decode_fwd outputs)
+ *   lse_parts  fp32 [num_ranks][batch][num_heads][s_q]
+ *   out        bf16 [batch][s_q][num_heads][d_v]
+ *   lse        fp32 [batch][num_heads][s_q]
+ * d_v is 512 (MLA path) or 128 (GQA path), else MLA_ERR_UNSUPPORTED.
+ * 1 <= num_ranks <= 64; batch, s_q, num_heads >= 1; every pointer device
+ * memory, 16-byte aligned, owned by the caller; out and lse must not overlap
+ * the inputs (else MLA_ERR_INVALID_ARG / undefined).  Enqueued on `stream`
+ * (NULL = legacy default); nothing is allocated.  Accumulates in fp32 and
+ * rounds once to bf16.
+ * ---------------------------------------------------------------------- */
+int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
+                             const void* o_parts, const float* lse_parts, void* out, float* lse,
+                             void* stream);
+
 /* Library ABI version (increments on any change of these declarations). */
 int mla_decode_version(void);
 

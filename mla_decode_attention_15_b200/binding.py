@@ -54,6 +54,7 @@ EXPORTED = (
     "mla_gqa_decode_combine",
     "mla_absorb_q",
     "mla_absorb_o",
+    "mla_decode_combine_ranks",
 )
 
 GQA_D_HEAD = 128
@@ -137,6 +138,9 @@ def lib() -> ctypes.CDLL:
         L.mla_gqa_decode_fwd.argtypes = [Q, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
         L.mla_gqa_decode_combine.restype = ctypes.c_int
         L.mla_gqa_decode_combine.argtypes = [Q, vp, vp, vp, vp, vp]
+        i32 = ctypes.c_int32
+        L.mla_decode_combine_ranks.restype = ctypes.c_int
+        L.mla_decode_combine_ranks.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         A = ctypes.POINTER(mla_absorb_dims)
         for name in ("mla_absorb_q", "mla_absorb_o"):
             getattr(L, name).restype = ctypes.c_int
@@ -442,3 +446,25 @@ def absorb_o(o: torch.Tensor, w_uv: torch.Tensor, out: Optional[torch.Tensor] = 
     _bf16_on(out, shape, "out", o.device)
     mla_absorb_o(make_absorb_dims(T, h), o, w_uv, out, None, stream)
     return out
+
+
+# ---------------------------------------------------------------- split-KV across ranks
+def mla_decode_combine_ranks(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor,
+                             lse: torch.Tensor, stream=None) -> None:
+    """o_parts bf16 [R, B, s_q, h, d_v], lse_parts fp32 [R, B, h, s_q] -> out
+    bf16 [B, s_q, h, d_v], lse fp32 [B, h, s_q]: the LSE-weighted merge of the
+    ranks' results (d_v 512 or 128)."""
+    _require(o_parts.dim() == 5 and o_parts.dtype == torch.bfloat16 and o_parts.is_contiguous(),
+             "o_parts must be contiguous bf16 [R, B, s_q, h, d_v]")
+    R, B, s_q, h, d_v = o_parts.shape
+    _require(lse_parts.dtype == torch.float32 and lse_parts.is_contiguous() and
+             tuple(lse_parts.shape) == (R, B, h, s_q), "lse_parts must be contiguous fp32 [R, B, h, s_q]")
+    _require(out.dtype == torch.bfloat16 and out.is_contiguous() and tuple(out.shape) == (B, s_q, h, d_v),
+             "out must be contiguous bf16 [B, s_q, h, d_v]")
+    _require(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, h, s_q),
+             "lse must be contiguous fp32 [B, h, s_q]")
+    for t in (lse_parts, out, lse):
+        _require(t.device == o_parts.device, "all tensors must be on %s" % o_parts.device)
+    _check(lib().mla_decode_combine_ranks(int(R), int(B), int(s_q), int(h), int(d_v), _ptr(o_parts),
+                                          _ptr(lse_parts), _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_decode_combine_ranks")

@@ -11,6 +11,7 @@
 
 #include "absorb_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "rank_combine.cuh"
 #include "mla_decode.h"
 #include "schedule.cuh"
 
@@ -18,7 +19,7 @@ namespace {
 
 using namespace mla;
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr int kMaxDevices = 64;
 
 int validate_dims(const mla_decode_dims* d) {
@@ -338,8 +339,8 @@ int launch_absorb(const mla_absorb_dims* d, const void* x, const void* w, void* 
         }
     }
     CUtensorMap wm, xm;
-    int rc = kKind == 0 ? make_weight_map(&wm, w, d->num_heads, kProjNope, kProjLatent, P::kWBoxRows)
-                        : make_weight_map(&wm, w, d->num_heads, kProjLatent, kProjVHead, P::kWBoxRows);
+    int rc = kKind == 0 ? make_weight_map(&wm, w, d->num_heads, kProjNope, kProjLatent, kProjTile)
+                        : make_weight_map(&wm, w, d->num_heads, kProjLatent, kProjVHead, kProjTile);
     if (rc != MLA_OK) return rc;
     rc = make_rows_map(&xm, x, d->tokens, d->num_heads, P::kInW);
     if (rc != MLA_OK) return rc;
@@ -349,8 +350,28 @@ int launch_absorb(const mla_absorb_dims* d, const void* x, const void* w, void* 
     p.status = status;
     p.T = d->tokens;
     p.heads = d->num_heads;
-    const dim3 grid(P::kChunks, d->num_heads, (d->tokens + kProjTokens - 1) / kProjTokens);
-    mla_absorb_kernel<kKind><<<grid, kProjThreads, P::kSmem, stream>>>(wm, xm, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P::kGridX, d->num_heads, (d->tokens + kProjTokens - 1) / kProjTokens);
+    cfg.blockDim = dim3(kProjThreads);
+    cfg.dynamicSmemBytes = P::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int na = 1;
+    if (kKind == 1) {  // the 4 K chunks of one head and token tile form a cluster
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = kProjSplitK;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        na = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, mla_absorb_kernel<kKind>, wm, xm, p) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -652,6 +673,33 @@ int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, v
     if (!aligned16(o) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
     if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return MLA_ERR_INVALID_ARG;
     return launch_absorb<1>(dims, o, w_uv, out, status, static_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
+                             const void* o_parts, const float* lse_parts, void* out, float* lse, void* stream) {
+    if (num_ranks < 1 || num_ranks > kRankCombineMaxRanks || batch < 1 || s_q < 1 || num_heads < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (d_v != kDv && d_v != ShapeGqa::kDv) return MLA_ERR_UNSUPPORTED;
+    const long long rows = (long long)batch * s_q * num_heads;
+    const long long blocks = (rows + kRankCombineWarps - 1) / kRankCombineWarps;
+    if (blocks > 0x7fffffffLL || rows * num_ranks * d_v > (1LL << 40)) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(out) || !aligned16(lse))
+        return MLA_ERR_INVALID_ARG;
+    RankCombineParams p;
+    p.o_parts = static_cast<const __nv_bfloat16*>(o_parts);
+    p.lse_parts = lse_parts;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.R = num_ranks;
+    p.B = batch;
+    p.s_q = s_q;
+    p.h = num_heads;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d_v == kDv)
+        mla_rank_combine_kernel<kDv><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
+    else
+        mla_rank_combine_kernel<ShapeGqa::kDv><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // extern "C"

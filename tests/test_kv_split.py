@@ -1,0 +1,220 @@
+"""Split-KV across ranks: the page split and causal assignment (host logic of
+mla_decode_attention_15_b200.kv_split), the merge oracle, a world-size-2 gloo
+run of the exchange on the CPU, and on one GPU the CUDA merge
+(mla_decode_combine_ranks) of R shard decodes run one after another.
+
+The merge oracle (oracle/merge.py) is pinned here against the whole-context
+decode oracle: merging the shards' exact results must reproduce it to fp64
+rounding, with causal s_q = 2 and with ranks that hold no page of a request."""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import helpers
+import oracle
+from oracle import merge
+from mla_decode_attention_15_b200 import _build, binding as bd, kv_split, workloads
+
+
+def test_page_ranges_tile_each_request():
+    for P in range(0, 41):
+        for R in range(1, 9):
+            ranges = [kv_split.page_range(P, R, r) for r in range(R)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == P
+            for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+                assert a1 == b0 and a0 <= a1
+            if P >= 1:
+                assert ranges[-1][1] - ranges[-1][0] >= 1  # the last rank holds the tail
+            sizes = [b - a for a, b in ranges]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        kv_split.page_range(4, 2, 2)
+
+
+def test_shard_reassembles_the_batch():
+    d = workloads.build(5, 1, 2, ("list", [1, 63, 64, 65, 700]), seed=61)
+    sl, bt = d["cache_seqlens"], d["block_table"]
+    for R in (1, 2, 3, 5):
+        parts = [kv_split.shard(sl, bt, R, r) for r in range(R)]
+        for b in range(5):
+            L = int(sl[b])
+            lens = [int(p[0][b]) for p in parts]
+            assert sum(lens) == L
+            assert all(x % 64 == 0 for x in lens[:-1])  # only the last rank has a partial page
+            pages = [int(x) for p in parts for x in p[1][b] if x >= 0]
+            assert pages == [int(x) for x in bt[b, :(L + 63) // 64]]
+    assert [kv_split.rank_causal(True, 3, r) for r in range(3)] == [False, False, True]
+    assert not kv_split.rank_causal(False, 3, 2)
+
+
+def _shard_oracle(d, R, causal):
+    outs, lses = [], []
+    for r in range(R):
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], R, r)
+        o, l = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], bt, sl, d["softmax_scale"],
+                                     causal=kv_split.rank_causal(causal, R, r))
+        outs.append(o)
+        lses.append(l)
+    return outs, lses
+
+
+@pytest.mark.parametrize("R,s_q,causal", [(2, 1, False), (3, 2, True), (4, 2, True)])
+def test_merge_oracle_reproduces_the_whole(oracle_mod, R, s_q, causal):
+    lens = [1, 2, 64, 65, 130, 257]  # requests shorter than R pages leave ranks empty
+    d = workloads.build(len(lens), s_q, 2, ("list", lens), seed=62 + R)
+    ow, lw = oracle_mod.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                       d["softmax_scale"], causal=causal)
+    outs, lses = _shard_oracle(d, R, causal)
+    assert any(np.isneginf(l).any() for l in lses)  # an empty shard took part
+    om, lm = merge.merge_partials(np.stack(outs), np.stack(lses))
+    np.testing.assert_allclose(om, ow, rtol=0, atol=1e-12)
+    fin = np.isfinite(lw)
+    assert np.array_equal(np.isneginf(lm), np.isneginf(lw))
+    np.testing.assert_allclose(lm[fin], lw[fin], rtol=0, atol=1e-12)
+
+
+def test_merge_oracle_special_cases():
+    o = np.arange(12, dtype=np.float64).reshape(1, 3, 4)
+    l = np.array([[0.5, -1.0, 2.0]])
+    om, lm = merge.merge_partials(o, l)  # one part: identity
+    np.testing.assert_array_equal(om, o[0])
+    np.testing.assert_array_equal(lm, l[0])
+    o2 = np.stack([o[0], 100 + o[0]])
+    l2 = np.stack([l[0], np.full(3, -np.inf)])  # an empty part weighs nothing
+    om, lm = merge.merge_partials(o2, l2)
+    np.testing.assert_array_equal(om, o[0])
+    np.testing.assert_array_equal(lm, l[0])
+    om, lm = merge.merge_partials(o2, np.full((2, 3), -np.inf))  # nothing visible anywhere
+    assert not om.any() and np.isneginf(lm).all()
+    l3 = np.stack([np.zeros(3), np.zeros(3)])  # equal shares: the mean, LSE + ln 2
+    om, lm = merge.merge_partials(o2, l3)
+    np.testing.assert_allclose(om, (o2[0] + o2[1]) / 2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lm, np.log(2.0), rtol=0, atol=1e-15)
+
+
+def _gloo_rank(rank, world, port, result_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        d = workloads.build(4, 2, 2, ("list", [3, 64, 200, 129]), seed=71)
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], world, rank)
+        o, l = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], bt, sl, d["softmax_scale"],
+                                     causal=kv_split.rank_causal(True, world, rank))
+        o_all = kv_split.gather(torch.from_numpy(o), None)
+        l_all = kv_split.gather(torch.from_numpy(l), None)
+        om, lm = merge.merge_partials(o_all.numpy(), l_all.numpy())
+        ow, lw = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                       d["softmax_scale"], causal=True)
+        ok = np.allclose(om, ow, rtol=0, atol=1e-12) and np.allclose(lm, lw, rtol=0, atol=1e-12)
+        with open("%s.%d" % (result_path, rank), "w") as f:
+            f.write("ok" if ok else "mismatch %g" % np.abs(om - ow).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_world2_exchange_and_merge(oracle_mod, tmp_path):
+    """Two CPU ranks: shard, decode with the oracle, all-gather over gloo
+    with kv_split.gather, merge; both ranks reproduce the whole decode."""
+    port = 29000 + os.getpid() % 1000
+    path = str(tmp_path / "res")
+    mp.start_processes(_gloo_rank, args=(2, port, path), nprocs=2, start_method="spawn", join=True)
+    for r in range(2):
+        assert open("%s.%d" % (path, r)).read() == "ok"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return bd.lib()
+
+
+def test_combine_ranks_rejections(lib):
+    f = lib.mla_decode_combine_ranks
+    good = (2, 4, 1, 16, 512, 0x1000, 0x2000, 0x3000, 0x4000, None)
+    for i, v in [(0, 0), (0, 65), (1, 0), (2, 0), (3, 0), (5, None), (6, 0x2004), (7, None), (8, 0x4008)]:
+        args = list(good)
+        args[i] = v
+        assert f(*args) == bd.MLA_ERR_INVALID_ARG, (i, v)
+    args = list(good)
+    args[4] = 576
+    assert f(*args) == bd.MLA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ GPU
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    _build.build()
+    bd.lib()
+    oracle.build()
+    return torch.device("cuda:0")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R,s_q,causal,heads", [(2, 1, False, 16), (3, 2, True, 16), (4, 2, True, 128),
+                                                (8, 1, False, 16)])
+def test_split_decode_then_merge_matches_whole_oracle(dev, R, s_q, causal, heads):
+    """R ranks emulated on one GPU, one after another (no kernel waits on
+    another): each decodes its shard with the C-ABI path, the stacked
+    results are merged by mla_decode_combine_ranks, and the merge is
+    compared with the whole-context oracle."""
+    lens = [1, 65, 640, 1000, 4096, 3000]
+    d = workloads.build(len(lens), s_q, heads, ("list", lens), seed=90 + R, sigma=0.5 if heads == 128 else 1.0)
+    B = len(lens)
+    q, kv = d["q"].to(dev), d["kv_cache"].to(dev)
+    o_parts = torch.empty(R, B, s_q, heads, 512, dtype=torch.bfloat16, device=dev)
+    l_parts = torch.empty(R, B, heads, s_q, dtype=torch.float32, device=dev)
+    for r in range(R):
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], R, r)
+        dec = bd.MlaDecoder(B, s_q, heads, kv.shape[0], bt.shape[1], kv_split.rank_causal(causal, R, r), 0, dev)
+        sl_d, bt_d = sl.to(dev), bt.to(dev)
+        dec.plan(sl_d)
+        o, l = dec(q, kv, bt_d, sl_d, d["softmax_scale"])
+        o_parts[r].copy_(o)
+        l_parts[r].copy_(l)
+        torch.cuda.synchronize()
+        assert dec.status() == 0
+    out = torch.empty(B, s_q, heads, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, heads, s_q, dtype=torch.float32, device=dev)
+    bd.mla_decode_combine_ranks(o_parts, l_parts, out, lse)
+    torch.cuda.synchronize()
+    ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                   d["softmax_scale"], causal=causal)
+    helpers.compare(out, lse, ro, rl)
+
+
+@pytest.mark.gpu
+def test_combine_ranks_kernel_against_merge_oracle(dev):
+    """The merge kernel alone on random partials (d_v 512 and 128), with
+    empty ranks and an all-empty row, against the fp64 merge oracle: one
+    bf16 rounding of an fp32 sum of R terms."""
+    g = torch.Generator().manual_seed(93)
+    for d_v in (512, 128):
+        R, B, s_q, h = 5, 3, 2, 16
+        o = (torch.randn(R, B, s_q, h, d_v, generator=g)).to(torch.bfloat16)
+        l = torch.randn(R, B, h, s_q, generator=g) * 4
+        l[1] = -float("inf")
+        l[:, 0, 3, 1] = -float("inf")
+        out = torch.empty(B, s_q, h, d_v, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(B, h, s_q, dtype=torch.float32, device=dev)
+        bd.mla_decode_combine_ranks(o.to(dev), l.to(dev), out, lse)
+        torch.cuda.synchronize()
+        rows = B * s_q * h
+        # merge oracle over flattened rows (b*s_q+s)*h+head; LSE rows in the same order
+        lo = l.permute(0, 1, 3, 2).reshape(R, rows).double().numpy()
+        om, lm = merge.merge_partials(o.reshape(R, rows, d_v).double().numpy(), lo)
+        got = out.reshape(rows, d_v).double().cpu().numpy()
+        mag = merge.merge_partials(np.abs(o.reshape(R, rows, d_v).double().numpy()), lo)[0]
+        tol = 2.0 ** -8 * np.abs(om) + 1e-5 * mag + 1e-30
+        assert (np.abs(got - om) <= tol).all()
+        gl = lse.permute(0, 2, 1).reshape(rows).double().cpu().numpy()
+        assert np.array_equal(np.isneginf(gl), np.isneginf(lm))
+        fin = np.isfinite(lm)
+        assert np.abs(gl[fin] - lm[fin]).max() <= 1e-5 * max(1.0, np.abs(lm[fin]).max())
+        assert not got[~fin].any()
