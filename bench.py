@@ -749,6 +749,13 @@ def run_absorb_bench(args):
                          "frac": achieved / hbm_peak, "tflops": 2 * T * h * 128 * 512 / (us * 1e-6) / 1e12}
         assert int(status.max()) == 0, "device status %#x" % int(status.max())
         cases.append({"case": name, "tokens": T, "heads": h, **res})
+    traffic = None
+    try:
+        tj = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic_absorb.json")))
+        if tj.get("kernel_source_hash") == kernel_source_hash():
+            traffic = sum(tj[k]["dram_bytes_read"] + tj[k]["dram_bytes_write"] for k in ("absorb_q", "absorb_o"))
+    except Exception:
+        traffic = None
     main_case = cases[1]
     us = main_case["absorb_q"]["us_per_call"] + main_case["absorb_o"]["us_per_call"]
     byt = main_case["absorb_q"]["algorithmic_bytes"] + main_case["absorb_o"]["algorithmic_bytes"]
@@ -761,7 +768,8 @@ def run_absorb_bench(args):
                    "l2": "61 layers of weights (244 MB / 2 GB) rotate: no flush"},
         "roofline": {"kernel": "mla_absorb_kernel", "bound": "hbm", "achieved": byt / (us * 1e-6) / 1e9,
                      "peak": hbm_peak, "unit": "GB/s", "frac": byt / (us * 1e-6) / 1e9 / hbm_peak,
-                     "peak_kind": peak_kind + " (copy bandwidth, burst)", "traffic": None},
+                     "peak_kind": peak_kind + " (copy bandwidth, burst)", "traffic": traffic,
+                     "traffic_note": "DRAM bytes of one absorb_q + one absorb_o launch (ncu, 1 pass)"},
         "cases": cases, "gpu_launches": 2 * layers * args.steps,
     }
     print(json.dumps(line), flush=True)

@@ -355,19 +355,11 @@ int launch_absorb(const mla_absorb_dims* d, const void* x, const void* w, void* 
     cfg.blockDim = dim3(kProjThreads);
     cfg.dynamicSmemBytes = P::kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    int na = 1;
-    if (kKind == 1) {  // the 4 K chunks of one head and token tile form a cluster
-        attr[1].id = cudaLaunchAttributeClusterDimension;
-        attr[1].val.clusterDim.x = kProjSplitK;
-        attr[1].val.clusterDim.y = 1;
-        attr[1].val.clusterDim.z = 1;
-        na = 2;
-    }
     cfg.attrs = attr;
-    cfg.numAttrs = na;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, mla_absorb_kernel<kKind>, wm, xm, p) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;

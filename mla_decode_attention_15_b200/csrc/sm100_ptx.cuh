@@ -101,32 +101,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* map, int c0, int c1,
                  : "memory");
 }
 
-// ---------------------------------------------------------------- clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// All threads of all CTAs of the cluster; release/acquire orders the shared
-// memory writes before it with the remote reads after it.
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// The address of the same shared-memory location in cluster CTA `rank`.
-__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // ---------------------------------------------------------------- dependent launch
 // Programmatic dependent launch: the next kernel in the stream may start once
 // every CTA of this one has called launch_dependents (or exited); it then
