@@ -72,6 +72,7 @@ struct ShapeMla {
     static constexpr int kVChunks = 4;     // d_v / 128: GEMM2 chunks of 128 rows
     static constexpr bool kPrefetchL2 = true;  // a page is one contiguous 72 KB block
     static constexpr int kStages = 2;          // 72 KB page stages
+    static constexpr bool kOneRun = true;      // a group's query columns are NG consecutive rows
     __host__ __device__ static constexpr int k_box(int c) { return c; }
     // first stage box of d_v chunk ch; the chunk's second box follows 8 KB on
     __host__ __device__ static constexpr int v_box(int ch) { return 2 * ch; }
@@ -88,6 +89,7 @@ struct ShapeGqa {
     static constexpr int kVChunks = 1;
     static constexpr bool kPrefetchL2 = false;  // a group's boxes are strided across the page
     static constexpr int kStages = 4;           // 40 KB page stages
+    static constexpr bool kOneRun = false;     // one run of 16 heads per new token
     __host__ __device__ static constexpr int k_box(int c) { return c; }
     __host__ __device__ static constexpr int v_box(int) { return 3; }
     __host__ __device__ static constexpr int col(int c, int kg, int kv_groups) {
@@ -219,6 +221,13 @@ struct FwdParams {
 __device__ __forceinline__ int item_col(int run_rows, int run_stride, int g, int q) {
     const int r = q / run_rows;
     return r * run_stride + g * run_rows + (q - r * run_rows);
+}
+// The same for a kernel instance: a cache shape whose groups are one run of
+// NG rows maps at compile time, without the division.
+template <int NG, class S>
+__device__ __forceinline__ int group_col(const FwdParams& p, int g, int q) {
+    if constexpr (S::kOneRun) return g * NG + q;
+    else return item_col(p.run_rows, p.run_stride, g, q);
 }
 
 struct CombineParams {
@@ -503,12 +512,14 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
         ok = wait_bounded(bar0 + 8 * kQEmpty, (q_it & 1) ^ 1, ctl);
         if (!ok) break;
         mbar_arrive_expect_tx(bar0 + 8 * kQFull, L::kQBytes);
+        const int run_rows = S::kOneRun ? NG : p.run_rows;
+        const int run_stride = S::kOneRun ? 0 : p.run_stride;
 #pragma unroll 1
-        for (int r = 0; r * p.run_rows < NG; ++r) {  // runs of query rows (one for MLA groups)
-            const int row0 = item.b * p.N + r * p.run_stride + item.g * p.run_rows;
+        for (int r = 0; r * run_rows < NG; ++r) {  // runs of query rows (one for MLA groups)
+            const int row0 = item.b * p.N + r * run_stride + item.g * run_rows;
 #pragma unroll 1
             for (int c = 0; c < S::kKBoxes; ++c)
-                tma_load_2d(q_s + c * L::kQBoxBytes + r * p.run_rows * 128, q_map, bar0 + 8 * kQFull,
+                tma_load_2d(q_s + c * L::kQBoxBytes + r * run_rows * 128, q_map, bar0 + 8 * kQFull,
                             c * L::kBoxCols, row0);
         }
         ++q_it;
@@ -746,7 +757,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         int lvis[W];                                      // visible length of each own column
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-            const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + par + 2 * i);
+            const int gc = group_col<NG, S>(p, item.g, c0g + par + 2 * i);
             int v = 0;
             if (gc < p.N) {
                 const int sq = gc / p.heads;
@@ -997,7 +1008,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             l_gt = gtg == n ? ls : l_gt;
         }
         {
-            const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + gtg);
+            const int gc = group_col<NG, S>(p, item.g, c0g + gtg);
             if (gtg < NGW && gc < p.N) {
                 const float lse = l_gt > 0.f ? (m_gt + log2f(l_gt)) * kLn2 : -INFINITY;
                 if (item.unsplit) {
@@ -1048,7 +1059,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     ok = wait_bounded(bar0 + 8 * kOutStaged, out_it & 1, ctl);
                     if (ok) {
                         // first query column of the pass; a pass stays within one run
-                        const int c0 = item_col(p.run_rows, p.run_stride, item.g, L::kOutRows * ps);
+                        const int c0 = group_col<NG, S>(p, item.g, L::kOutRows * ps);
                         if (f32) {
                             if (item.slot >= 0)
                                 bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * S::kDv,
@@ -1089,7 +1100,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     if (f32) {
                         if (item.slot >= 0) p.opart[((size_t)item.slot * NG + c0g + n) * S::kDv + d] = v;
                     } else {
-                        const int gc = item_col(p.run_rows, p.run_stride, item.g, c0g + n);
+                        const int gc = group_col<NG, S>(p, item.g, c0g + n);
                         if (gc < p.N) p.out[((size_t)item.b * p.N + gc) * S::kDv + d] = __float2bfloat16_rn(v);
                     }
                 }
@@ -1238,7 +1249,8 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     }
     const int b = bg / p.Hg;
     const int g = bg - b * p.Hg;
-    const int gc = item_col(p.run_rows, p.run_stride, g, n);
+    // one run (MLA groups): no division
+    const int gc = p.run_stride == 0 ? g * p.run_rows + n : item_col(p.run_rows, p.run_stride, g, n);
     if (gc >= p.N) return;
     const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
     const int base = __ldg(info + 0);
