@@ -7,6 +7,7 @@ The merge oracle (oracle/merge.py) is pinned here against the whole-context
 decode oracle: merging the shards' exact results must reproduce it to fp64
 rounding, with causal s_q = 2 and with ranks that hold no page of a request."""
 import ctypes
+import datetime
 import os
 
 import numpy as np
@@ -218,3 +219,41 @@ def test_combine_ranks_kernel_against_merge_oracle(dev):
         fin = np.isfinite(lm)
         assert np.abs(gl[fin] - lm[fin]).max() <= 1e-5 * max(1.0, np.abs(lm[fin]).max())
         assert not got[~fin].any()
+
+
+def _nccl_one_rank(rank, port, result_path):
+    """KvSplitDecoder end to end in a one-rank NCCL group: local decode,
+    NCCL all-gather, CUDA merge (a single rank waits on no other)."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    msg = "not run"
+    try:
+        dev = torch.device("cuda:0")
+        d = workloads.build(3, 2, 16, ("list", [1, 65, 3000]), seed=95)
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], 1, 0)
+        dec = kv_split.KvSplitDecoder(3, 2, 16, d["kv_cache"].shape[0], bt.shape[1], causal=True, device=dev)
+        sl_d, bt_d = sl.to(dev), bt.to(dev)
+        dec.plan(sl_d)
+        out, lse = dec(d["q"].to(dev), d["kv_cache"].to(dev), bt_d, sl_d, d["softmax_scale"])
+        torch.cuda.synchronize()
+        assert dec.dec.status() == 0
+        ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                       d["softmax_scale"], causal=True)
+        helpers.compare(out, lse, ro, rl)
+        msg = "ok"
+    except Exception as e:  # reported to the parent through the result file
+        msg = "error: %r" % (e,)
+    finally:
+        dist.destroy_process_group()
+        with open(result_path, "w") as f:
+            f.write(msg)
+
+
+@pytest.mark.gpu
+def test_kv_split_decoder_one_rank_nccl(dev, tmp_path):
+    port = 30000 + os.getpid() % 1000
+    path = str(tmp_path / "nccl_res")
+    mp.start_processes(_nccl_one_rank, args=(port, path), nprocs=1, start_method="spawn", join=True)
+    assert open(path).read() == "ok"
