@@ -233,9 +233,10 @@ def aggregate_over_ranks(times_ms, kv_bytes: float, device) -> tuple:
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample_rate(d, w, budget_s: float, max_requests=None):
+def oracle_sample_rate(d, w, budget_s: float, max_requests=None, collect=None):
     """Times the fp64 oracle on whole requests (all heads x s_q rows of each)
-    until about budget_s of wall time; returns (GB/s of KV, seconds, sample text, cores)."""
+    until about budget_s of wall time; returns (GB/s of KV, seconds, sample text, cores).
+    With ``collect`` (a list), appends (rows, out, lse) of every request done."""
     import oracle
     oracle.build()
     cores = oracle.max_threads()
@@ -247,9 +248,11 @@ def oracle_sample_rate(d, w, budget_s: float, max_requests=None):
     for b in range(B):
         rows = list(range(b * rows_per_req, (b + 1) * rows_per_req))
         t = time.perf_counter()
-        oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
-                              d["softmax_scale"], causal=d["causal"], rows=rows)
+        res = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                    d["softmax_scale"], causal=d["causal"], rows=rows)
         elapsed += time.perf_counter() - t
+        if collect is not None:
+            collect.append((rows, res[0], res[1]))
         done_bytes += int(max(int(d["cache_seqlens"][b]), 0)) * 576 * 2
         n_req += 1
         if elapsed >= budget_s:
@@ -257,6 +260,30 @@ def oracle_sample_rate(d, w, budget_s: float, max_requests=None):
     sample = "%d of %d requests (all %d heads x s_q %d rows each, %d KV tokens)" % (
         n_req, w.batch, w.heads, w.s_q, done_bytes // 1152)
     return done_bytes / elapsed / 1e9, elapsed, sample, cores
+
+
+def bench_parity(done, out_rows, lse_rows):
+    """Outputs of the timed launch configuration against the oracle rows the
+    CPU baseline computed: max|err| relative to max|ref|, RMSE (with the
+    bf16 rounding floor of the exact result), LSE relative error."""
+    import numpy as np
+    if not done:
+        return None
+    rows = np.concatenate([np.asarray(r) for r, _, _ in done])
+    ref = np.concatenate([o for _, o, _ in done])
+    ref_l = np.concatenate([l for _, _, l in done])
+    got = out_rows[rows].astype(np.float64)
+    got_l = lse_rows[rows].astype(np.float64)
+    err = got - ref
+    bf = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+    fin = np.isfinite(ref_l)
+    return {"rows": int(rows.size), "oracle": "fp64",
+            "max_abs_err_over_max_ref": float(np.abs(err).max() / max(np.abs(ref).max(), 1e-30)),
+            "rmse": float(np.sqrt(np.mean(err ** 2))),
+            "bf16_floor_rmse": float(np.sqrt(np.mean((bf - ref) ** 2))),
+            "lse_rel_err": float((np.abs(got_l[fin] - ref_l[fin]) / np.maximum(1.0, np.abs(ref_l[fin]))).max())
+            if fin.any() else 0.0,
+            "lse_neginf_match": bool(np.array_equal(np.isneginf(got_l), np.isneginf(ref_l)))}
 
 
 def run_reference(args, w):
@@ -419,6 +446,12 @@ def run_ours(args, w):
     status = bd.mla_decode_get_status(sched)
     assert status == 0, "device status %#x" % status
     del g_step, g_dec
+    # One more full step (outside the timed region): its outputs are checked
+    # against the oracle rows that the CPU baseline computes.
+    step()
+    torch.cuda.synchronize()
+    out_check = out.float().cpu().numpy().reshape(-1, 512)
+    lse_check = lse.cpu().numpy().transpose(0, 2, 1).reshape(-1)  # rows (b*s_q+s)*h+head
 
     (ms_step, kernel_ms), total_kv = aggregate_over_ranks([ms_step, kernel_ms], byt["kv"], dev)
 
@@ -438,10 +471,13 @@ def run_ours(args, w):
     roof_us_meas = max(byt["total"] / (hbm_peak * 1e9), flops / (tf_peak * 1e12)) * 1e6
     roof_us_nom = max(byt["total"] / (NOMINAL_HBM_GBS * 1e9), flops / (tf_peak * 1e12)) * 1e6
     cpu = None
+    parity = None
     if world == 1 and not args.no_cpu_baseline:
-        r, t, sample, cores = oracle_sample_rate(d, w, budget_s=15.0)
+        done = []
+        r, t, sample, cores = oracle_sample_rate(d, w, budget_s=15.0, collect=done)
         cpu = {"value": r, "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": sample + " (%.1f s)" % t}
+        parity = bench_parity(done, out_check, lse_check)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": ms_step * 1e3,
@@ -455,6 +491,7 @@ def run_ours(args, w):
                                   "at_8tbs": roof_us_nom / (ms_step * 1e3)},
         "roofline": kernel_roofline(byt, flops, kernel_ms, hbm_peak, tf_peak, peak_kind, traffic),
         "cpu_baseline": cpu,
+        "parity": parity,
         "e2e": e2e,
         "clocks": clocks.summary(wall0, wall1),
         "gpu_launches": 3 * args.steps,

@@ -185,6 +185,26 @@ def test_repeat_runs_are_bitwise_identical(dev):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("heads,s_q", [(16, 2), (128, 2)])
+def test_poisoned_workspace_and_outputs(dev, heads, s_q):
+    """Workspace, out and lse start as NaN: the result still matches the
+    oracle, so every output element is written and no split partial (nor the
+    padding between partial slots) is read before it is written."""
+    lens = [1, 64, 1000, 5000, 130, 0, 4099, 3000]
+    d = workloads.build(len(lens), s_q, heads, ("list", lens), seed=777 + heads, causal=True)
+    g = to_dev(d, dev)
+    dec = bd.MlaDecoder(len(lens), s_q, heads, g["kv_cache"].shape[0], g["block_table"].shape[1], True, 148, dev)
+    dec.workspace.view(torch.float32).fill_(float("nan"))
+    dec.out.fill_(float("nan"))
+    dec.lse.fill_(float("nan"))
+    dec.plan(g["cache_seqlens"])
+    out, lse = dec(g["q"], g["kv_cache"], g["block_table"], g["cache_seqlens"], g["softmax_scale"])
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    ro, rl = ref(d)
+    helpers.compare(out, lse, ro, rl)
+
+
 def test_explicit_combine_matches_fused_launch(dev):
     d = workloads.build(3, 1, 16, ("list", [5000, 64, 2222]), seed=71)
     o1, l1, _ = run_gpu(d, dev, num_sms=16)
