@@ -99,3 +99,31 @@ class KvSplitDecoder:
         l_all = gather(l, self.group)
         bd.mla_decode_combine_ranks(o_all, l_all, self.out, self.lse)
         return self.out, self.lse
+
+
+class KvSplitGqaDecoder:
+    """The same split for the GQA path over a group-expanded cache: every
+    rank holds a contiguous part of each request's pages (all KV groups of a
+    token live in one row), decodes it with ``GqaDecoder``, and the ranks
+    merge their 128-wide outputs by LSE."""
+
+    def __init__(self, batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
+                 causal: bool = False, group=None, device: Optional[torch.device] = None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.dec = bd.GqaDecoder(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq,
+                                 rank_causal(causal, self.world, self.rank), device=device)
+        dev = self.dec.device
+        h = self.dec.dims.num_q_heads
+        self.out = torch.empty(batch, s_q, h, bd.GQA_D_HEAD, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(batch, h, s_q, dtype=torch.float32, device=dev)
+
+    def plan(self, local_seqlens: torch.Tensor) -> None:
+        self.dec.plan(local_seqlens)
+
+    def __call__(self, q, kv_local, block_table_local, seqlens_local,
+                 softmax_scale: float) -> Tuple[torch.Tensor, torch.Tensor]:
+        o, l = self.dec(q, kv_local, block_table_local, seqlens_local, softmax_scale)
+        bd.mla_decode_combine_ranks(gather(o, self.group), gather(l, self.group), self.out, self.lse)
+        return self.out, self.lse

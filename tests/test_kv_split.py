@@ -129,6 +129,38 @@ def test_gloo_world2_exchange_and_merge(oracle_mod, tmp_path):
         assert open("%s.%d" % (path, r)).read() == "ok"
 
 
+def _gloo_rank_gqa(rank, world, port, result_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        d = workloads.build_gqa(3, 2, 2, ("list", [2, 129, 300]), seed=72, causal=True)
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], world, rank)
+        o, l = oracle.gqa_oracle_fwd(d["q"], d["kv_cache"], bt, sl, d["softmax_scale"], d["groups"],
+                                     causal=kv_split.rank_causal(True, world, rank))
+        om, lm = merge.merge_partials(kv_split.gather(torch.from_numpy(o), None).numpy(),
+                                      kv_split.gather(torch.from_numpy(l), None).numpy())
+        ow, lw = oracle.gqa_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                       d["softmax_scale"], d["groups"], causal=True)
+        fin = np.isfinite(lw)
+        ok = (np.allclose(om, ow, rtol=0, atol=1e-12) and np.array_equal(np.isneginf(lm), np.isneginf(lw))
+              and np.allclose(lm[fin], lw[fin], rtol=0, atol=1e-12))
+        with open("%s.%d" % (result_path, rank), "w") as f:
+            f.write("ok" if ok else "mismatch %g" % np.abs(om - ow).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_world2_gqa_path(oracle_mod, tmp_path):
+    """The same exchange for the GQA path: two CPU ranks, GQA oracle on each
+    shard (causal s_q 2, 2 KV groups), gather over gloo, merge = whole."""
+    port = 29000 + (os.getpid() + 500) % 1000
+    path = str(tmp_path / "res_gqa")
+    mp.start_processes(_gloo_rank_gqa, args=(2, port, path), nprocs=2, start_method="spawn", join=True)
+    for r in range(2):
+        assert open("%s.%d" % (path, r)).read() == "ok"
+
+
 @pytest.fixture(scope="module")
 def lib():
     _build.build()
@@ -187,6 +219,37 @@ def test_split_decode_then_merge_matches_whole_oracle(dev, R, s_q, causal, heads
     torch.cuda.synchronize()
     ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
                                    d["softmax_scale"], causal=causal)
+    helpers.compare(out, lse, ro, rl)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R,groups", [(2, 2), (3, 8)])
+def test_gqa_split_decode_then_merge_matches_whole_oracle(dev, R, groups):
+    """The GQA path split over R emulated ranks (causal s_q 2): shard decodes
+    through the C ABI one after another, merged by mla_decode_combine_ranks
+    (d_v 128), against the whole-context GQA oracle."""
+    lens = [1, 65, 640, 3000]
+    d = workloads.build_gqa(len(lens), 2, groups, ("list", lens), seed=96 + R, causal=True)
+    B, h = len(lens), 16 * groups
+    q, kv = d["q"].to(dev), d["kv_cache"].to(dev)
+    o_parts = torch.empty(R, B, 2, h, 128, dtype=torch.bfloat16, device=dev)
+    l_parts = torch.empty(R, B, h, 2, dtype=torch.float32, device=dev)
+    for r in range(R):
+        sl, bt = kv_split.shard(d["cache_seqlens"], d["block_table"], R, r)
+        dec = bd.GqaDecoder(B, 2, groups, kv.shape[0], bt.shape[1], kv_split.rank_causal(True, R, r), 0, dev)
+        sl_d, bt_d = sl.to(dev), bt.to(dev)
+        dec.plan(sl_d)
+        o, l = dec(q, kv, bt_d, sl_d, d["softmax_scale"])
+        o_parts[r].copy_(o)
+        l_parts[r].copy_(l)
+        torch.cuda.synchronize()
+        assert dec.status() == 0
+    out = torch.empty(B, 2, h, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, h, 2, dtype=torch.float32, device=dev)
+    bd.mla_decode_combine_ranks(o_parts, l_parts, out, lse)
+    torch.cuda.synchronize()
+    ro, rl = oracle.gqa_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                   d["softmax_scale"], groups, causal=True)
     helpers.compare(out, lse, ro, rl)
 
 
