@@ -468,3 +468,17 @@ def mla_decode_combine_ranks(o_parts: torch.Tensor, lse_parts: torch.Tensor, out
     _check(lib().mla_decode_combine_ranks(int(R), int(B), int(s_q), int(h), int(d_v), _ptr(o_parts),
                                           _ptr(lse_parts), _ptr(out), _ptr(lse), _stream(stream)),
            "mla_decode_combine_ranks")
+
+
+def absorbed_mla_decode(q_in: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor, kv_cache: torch.Tensor,
+                        block_table: torch.Tensor, cache_seqlens: torch.Tensor, softmax_scale: float,
+                        decoder: "MlaDecoder", stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One absorbed-MLA decode step for one layer: q_in [B, s_q, h, 192]
+    (each head's 128-wide part, then its RoPE part) -> the latent query
+    (mla_absorb_q), attention over the latent cache (mla_decode_fwd with
+    ``decoder``'s plan, already built by ``decoder.plan``), then the output
+    projection (mla_absorb_o).  Returns (out [B, s_q, h, 128] bf16, lse
+    [B, h, s_q] fp32: the attention's log-sum-exp)."""
+    q_lat = absorb_q(q_in, w_uk, stream=stream)
+    o_lat, lse = decoder(q_lat, kv_cache, block_table, cache_seqlens, softmax_scale, stream)
+    return absorb_o(o_lat, w_uv, stream=stream), lse
