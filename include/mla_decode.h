@@ -57,7 +57,7 @@ extern "C" {
 /* return codes */
 #define MLA_OK 0
 #define MLA_ERR_INVALID_ARG (-1)  /* null or misaligned pointer, negative size, bad dims */
-#define MLA_ERR_UNSUPPORTED (-2)  /* page_size != 64, d_qk != 576, d_v != 512, heads*s_q > 256 */
+#define MLA_ERR_UNSUPPORTED (-2)  /* page_size != 64, d_qk != 576, d_v != 512, s_q not 1 or 2, heads*s_q > 256 */
 #define MLA_ERR_CUDA (-3)         /* a CUDA runtime/driver call or launch failed */
 #define MLA_ERR_BAD_SCHEDULE (-4) /* schedule buffer was not built for these dims */
 #define MLA_ERR_SCRATCH_TOO_SMALL (-5) /* mla_decode_fwd_noalloc: the request needs more than its built-in scratch */
@@ -78,10 +78,17 @@ extern "C" {
  * MLA_STATUS_TIMEOUT through mla_decode_get_status, its outputs are undefined,
  * and the device stays usable. */
 #define MLA_FLAG_TEST_STALL 0x2
+/* `out` is fp32 [batch][s_q][num_heads][d_v] instead of bf16: the result as
+ * accumulated, before any rounding to bf16.  For a caller that feeds the
+ * output to an fp32 consumer (for example the output projection, or an
+ * exchange of partial results between GPUs), and for accuracy checks of the
+ * accumulation itself.  Applies to mla_decode_fwd, mla_decode_combine and
+ * the GQA-path calls; pass the same flags to both when combining separately. */
+#define MLA_FLAG_FP32_OUT 0x4
 
 typedef struct mla_decode_dims {
     int32_t batch;              /* B >= 1 */
-    int32_t s_q;                /* new tokens per request, >= 1 (1 or 2 in the workloads) */
+    int32_t s_q;                /* new tokens per request: 1 or 2 (else MLA_ERR_UNSUPPORTED) */
     int32_t num_heads;          /* h >= 1, h * s_q <= 256 */
     int32_t num_blocks;         /* pages in the pool */
     int32_t max_blocks_per_seq; /* row stride of block_table */
@@ -126,7 +133,7 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* cac
  *                ceil(L_b / 64) entries of row b are read
  *   cache_seqlens int32 [batch]: L_b, the cached length including the s_q new tokens
  *   softmax_scale scale applied to q.k (e.g. 192^-0.5)
- *   out          bf16 [batch][s_q][num_heads][512]
+ *   out          bf16 [batch][s_q][num_heads][512] (fp32 with MLA_FLAG_FP32_OUT)
  *   lse          fp32 [batch][num_heads][s_q]  (natural log; -inf if nothing is visible)
  *   schedule     from mla_decode_get_schedule with the same dims and lengths
  *   workspace    mla_decode_workspace_bytes(dims) bytes, no initialisation needed

@@ -31,6 +31,7 @@ MLA_STATUS_SMEM_ALIGN = 0x10
 
 MLA_FLAG_NO_COMBINE = 0x1
 MLA_FLAG_TEST_STALL = 0x2
+MLA_FLAG_FP32_OUT = 0x4
 
 PAGE_SIZE = 64
 D_QK = 576
@@ -240,22 +241,26 @@ class MlaDecoder:
 
     ``plan(cache_seqlens)`` builds the split-KV schedule (once per decode step);
     ``__call__`` runs the decode kernel + combine and returns (out, lse).
+    With ``fp32_out`` the output is fp32 (MLA_FLAG_FP32_OUT): the result before
+    any rounding to bf16.
     """
 
     def __init__(self, batch: int, s_q: int, num_heads: int, num_blocks: int,
                  max_blocks_per_seq: int, causal: bool = False, num_sms: int = 0,
-                 device: Optional[torch.device] = None):
+                 device: Optional[torch.device] = None, fp32_out: bool = False):
         self.device = torch.device(device or "cuda")
         if num_sms == 0:
             num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
-        self.dims = make_dims(batch, s_q, num_heads, num_blocks, max_blocks_per_seq, causal, num_sms)
+        self.dims = make_dims(batch, s_q, num_heads, num_blocks, max_blocks_per_seq, causal, num_sms,
+                              MLA_FLAG_FP32_OUT if fp32_out else 0)
         sb = mla_decode_schedule_bytes(self.dims)
         wb = mla_decode_workspace_bytes(self.dims)
         if sb == 0 or wb == 0:
             raise MlaDecodeError(MLA_ERR_INVALID_ARG, "MlaDecoder dims")
         self.schedule = torch.empty(sb, dtype=torch.uint8, device=self.device)
         self.workspace = torch.empty(wb, dtype=torch.uint8, device=self.device)
-        self.out = torch.empty(batch, s_q, num_heads, D_V, dtype=torch.bfloat16, device=self.device)
+        self.out = torch.empty(batch, s_q, num_heads, D_V, dtype=torch.float32 if fp32_out else torch.bfloat16,
+                               device=self.device)
         self.lse = torch.empty(batch, num_heads, s_q, dtype=torch.float32, device=self.device)
 
     def check_inputs(self, q, kv_cache, block_table, cache_seqlens) -> None:

@@ -130,6 +130,21 @@ struct FwdWarps {
                                      kRegsLaunch * kThreads,
                   "register split exceeds the launch allocation");
 };
+// P as two bf16 terms.  GEMM2 takes bf16 operands, and rounding P to bf16
+// costs up to 2^-9 of each weight, which shows in the fp32 result of peaked
+// rows (one token far above the rest).  Where the query group is at most 32
+// columns wide, the softmax writes P = hi + lo (hi = bf16(P), lo = bf16(P -
+// hi), together within 2^-17 of P) as 2 x NG columns of P^T, and GEMM2
+// accumulates both halves of O^T in one MMA of N = 2 x NG: an MMA of N <= 64
+// occupies the tensor pipe as long as one of N = 16, so the second term costs
+// no MMA time.  The epilogue adds the halves.  64-column groups (N = 128 would
+// double GEMM2's pipe time and O^T would need all of TMEM) keep one bf16 term;
+// so does the GQA shape.
+template <int NG, class S>
+struct PSplit {
+    static constexpr bool kOn = NG <= 32 && S::kVChunks == 4;
+    static constexpr int kNP = kOn ? 2 * NG : NG;  // P^T columns = GEMM2 N = O^T columns per d_v chunk
+};
 // Rescale O only when the running max grows by > 2^8.  Measured on B200
 // (bs16 x 64K decode kernel): an exact running max (rescale on any growth)
 // costs 6% (202.2 -> 214.4 us); with O normalised by the sum of the
@@ -203,13 +218,14 @@ struct FwdParams {
     const int32_t* block_table;
     const int32_t* seqlens;
     const uint8_t* kv;  // page pool base (for L2 prefetch)
-    __nv_bfloat16* out;
+    void* out;          // bf16 rows, or fp32 rows when out_f32
     float* lse;
     float* opart;  // [slots][NG][512]
     float* lpart;  // [slots][NG]
     int32_t* status;
     int s_q, heads, N, num_blocks, max_blocks, causal;
     int G, BG, Hg, slots_cap;
+    int out_f32;       // MLA_FLAG_FP32_OUT: final rows are written as fp32
     float scale_log2;  // softmax_scale * log2(e)
     int test_stall;    // MLA_FLAG_TEST_STALL: leave the first page unloaded
     // Query columns of a work item: runs of run_rows consecutive rows, run r
@@ -234,11 +250,12 @@ struct CombineParams {
     const int32_t* sched;
     const float* opart;
     const float* lpart;
-    __nv_bfloat16* out;
+    void* out;  // bf16 rows, or fp32 rows when out_f32
     float* lse;
     int32_t* status;
     int s_q, heads, N, NG, Hg, G, BG, slots_cap;
     int run_rows, run_stride;
+    int out_f32;
 };
 
 // ------------------------------------------------------------------ layout
@@ -252,7 +269,8 @@ struct FwdSmem {
     static constexpr int kStageBytes = kBoxes * kBoxBytes;    // 72 KB: one MLA page
     static constexpr int kQBoxBytes = NG * 128;               // NG rows x 64 cols
     static constexpr int kQBytes = S::kKBoxes * kQBoxBytes;
-    static constexpr int kPBytes = kPage * NG * 2;            // P^T of one page, bf16
+    static constexpr int kNP = PSplit<NG, S>::kNP;            // P^T columns (hi and lo halves when split)
+    static constexpr int kPBytes = kPage * kNP * 2;           // P^T of one page, bf16
     // P^T of a page is written over the page's own RoPE box (box 8): only
     // GEMM1 reads that box, S^T is complete before the softmax writes P^T, and
     // the stage is refilled only after the page's GEMM2 has read P^T.  So P^T
@@ -282,10 +300,10 @@ struct FwdSmem {
     static constexpr int kAlignSlack = kBytes + 1024 <= 227 * 1024 ? 1024 : 0;
     static constexpr int kAlloc = kBytes + kAlignSlack;
     // TMEM columns: S^T buffer i, chain c at kSCol + (i*G1<NG>::kIssuers + c)*NG;
-    // O^T d_v chunk c at kOCol + c*NG.
+    // O^T d_v chunk c at kOCol + c*kNP (hi half, then the lo half when split).
     static constexpr int kSCol = 0;
     static constexpr int kOCol = 2 * G1<NG>::kIssuers * NG;
-    static constexpr int kTmemUsed = kOCol + S::kVChunks * NG;
+    static constexpr int kTmemUsed = kOCol + S::kVChunks * kNP;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
     static_assert(kTmemUsed <= 512, "TMEM budget");
@@ -293,6 +311,7 @@ struct FwdSmem {
                   "swizzle atoms need 1 KB alignment");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
     static_assert(kStages >= 2 && kStages <= kMaxStages, "stage count");
+    static_assert(!PSplit<NG, S>::kOn || kOutRows > 0, "split P is summed by the staged epilogue");
 };
 
 enum Bar {
@@ -648,8 +667,9 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     constexpr int kIssuers = FwdWarps<NG, S>::kG2Issuers;
     constexpr int kChunksPer = S::kVChunks / kIssuers;  // d_v chunks of 128 per issuer
     using L = FwdSmem<NG, S>;
-    constexpr uint32_t kIdescO = idesc_bf16_f32(128, NG, 1, 1);
-    constexpr uint32_t kPSwizzle = NG == 16 ? kSwizzle32 : NG == 32 ? kSwizzle64 : kSwizzle128;
+    constexpr int NP = L::kNP;
+    constexpr uint32_t kIdescO = idesc_bf16_f32(128, NP, 1, 1);
+    constexpr uint32_t kPSwizzle = NP == 16 ? kSwizzle32 : NP == 32 ? kSwizzle64 : kSwizzle128;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t p_s = kv_s + L::kPInStage;  // P^T of stage 0
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
@@ -662,7 +682,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     Tracer tracer_(issuer == 0 ? 2 : 0, issuer == 0);
 #endif
     const uint64_t a_desc0 = smem_desc(kv_s, L::kBoxBytes, 1024, kSwizzle128);
-    const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NG * 2, kPSwizzle);
+    const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NP * 2, kPSwizzle);
     while (ok && it.next(p, bginfo, item)) {
         for (int j = item.p0; j < item.p1; ++j) {
             const int st = s_it % L::kStages;  // KV stage of the page (holds its P^T)
@@ -680,12 +700,12 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
             const uint64_t b_st = b_desc0 + ((st * L::kStageBytes) >> 4);
 #pragma unroll
             for (int k = 0; k < kPage / 16; ++k) {
-                const uint64_t b = b_st + ((k * 16 * NG * 2) >> 4);
+                const uint64_t b = b_st + ((k * 16 * NP * 2) >> 4);
 #pragma unroll
                 for (int cc = 0; cc < kChunksPer; ++cc) {
                     const int ch = issuer * kChunksPer + cc;
                     const uint64_t a = a_st + ((S::v_box(ch) * L::kBoxBytes + k * 2048) >> 4);
-                    umma_f16(tmem + L::kOCol + ch * NG, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
+                    umma_f16(tmem + L::kOCol + ch * NP, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
                 }
             }
             issued = true;
@@ -708,6 +728,8 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                             uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
     using L = FwdSmem<NG, S>;
     using Wp = FwdWarps<NG, S>;
+    constexpr bool kSplit = PSplit<NG, S>::kOn;           // P^T = [hi | lo] (2 x NG columns)
+    constexpr int NP = L::kNP;
     constexpr int NGW = Wp::kGroupCols;                   // query columns of this warp's group
     constexpr int W = NGW / 2;                            // own columns per thread
     const int warp = threadIdx.x >> 5;
@@ -733,12 +755,14 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     const int red_i = half_reduced_index<NGW>(lane);
     const int red_col = c0g + par + 2 * red_i;            // column whose reduction this thread holds
     const bool red_w = half_reduced_writer<NGW>(lane);
-    // P^T row: NG bf16 positions; the group owns positions c0g .. c0g+NGW-1,
-    // parity-major inside (own columns of parity par at c0g + par*W ..).
-    constexpr int kChunks = NG * 2 / 16;                  // 16-byte chunks per P^T row
-    constexpr int kMyChunks = NGW / 16;                   // chunks of one thread
+    // P^T row: NP bf16 positions; the group owns positions c0g .. c0g+NGW-1,
+    // parity-major inside (own columns of parity par at c0g + par*W ..); with
+    // a split P the lo terms follow at NG + the same positions.
+    constexpr int kChunks = NP * 2 / 16;                  // 16-byte chunks per P^T row
+    constexpr int kMyChunks = NGW / 16;                   // chunks of one thread (per term)
+    constexpr int kLoChunk = NG * 2 / 16;                 // chunk offset of the lo terms
     const int chunk0 = cg * (NGW / 8) + par * kMyChunks;
-    const int swz = ((row * NG * 2) >> 7) & (kChunks - 1);
+    const int swz = ((row * NP * 2) >> 7) & (kChunks - 1);
 #ifdef MLA_TRACE
     Tracer tracer_(3);
     const bool tr = (gt == 0);
@@ -837,19 +861,35 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 #pragma unroll
             for (int i = 0; i < W; ++i) e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m_own[i]);
             const int pb = s_it & 1;                      // P^T handoff barriers
-            uint8_t* rowp = pbuf + (s_it % L::kStages) * L::kStageBytes + row * (NG * 2);  // the page's stage
+            uint8_t* rowp = pbuf + (s_it % L::kStages) * L::kStageBytes + row * (NP * 2);  // the page's stage
             auto store_p = [&](const float (&ev)[W]) {
                 uint32_t packed[W / 2];
+                uint32_t packed_lo[kSplit ? W / 2 : 1];
 #pragma unroll
                 for (int i = 0; i < W; i += 2) {
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(ev[i], ev[i + 1]);
                     packed[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    if constexpr (kSplit) {
+                        // P - hi is exact in fp32 (hi is P rounded to 8 bits), so
+                        // lo carries the next 8 bits of P.
+                        const float2 hf = __bfloat1622float2(h2);
+                        const __nv_bfloat162 l2 = __floats2bfloat162_rn(ev[i] - hf.x, ev[i + 1] - hf.y);
+                        packed_lo[i / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+                    }
                 }
 #pragma unroll
                 for (int c = 0; c < kMyChunks; ++c) {
                     const int chunk = chunk0 + c;
                     *reinterpret_cast<uint4*>(rowp + ((chunk ^ swz) * 16)) =
                         make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                }
+                if constexpr (kSplit) {
+#pragma unroll
+                    for (int c = 0; c < kMyChunks; ++c) {
+                        const int chunk = kLoChunk + chunk0 + c;
+                        *reinterpret_cast<uint4*>(rowp + ((chunk ^ swz) * 16)) = make_uint4(
+                            packed_lo[4 * c], packed_lo[4 * c + 1], packed_lo[4 * c + 2], packed_lo[4 * c + 3]);
+                    }
                 }
             };
             ok = wait_warp(bar0 + 8 * (kPEmpty0 + pb), ((s_it >> 1) & 1) ^ 1, ctl);
@@ -900,7 +940,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
 #pragma unroll
                 for (int i = 0; i < W; ++i) {
                     l_own[i] += e[i];
-                    lq_own[i] += bf16_round(e[i]);
+                    if constexpr (!kSplit) lq_own[i] += bf16_round(e[i]);
                 }
             } else {
                 // Slow path: the group's exact page maxima are in rb; move the
@@ -926,7 +966,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     const float m = par ? m_all[2 * i + 1] : m_all[2 * i];
                     e[i] = (x[i] == -INFINITY) ? 0.f : ex2_approx(x[i] - m);
                     l_own[i] = l_own[i] * a + e[i];
-                    lq_own[i] = lq_own[i] * a + bf16_round(e[i]);
+                    if constexpr (!kSplit) lq_own[i] = lq_own[i] * a + bf16_round(e[i]);
                 }
                 // scale_any is the same for the group's four warps (same maxima).
                 if (scale_any) {
@@ -942,7 +982,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
-                    for (int ch = 0; ch < S::kVChunks; ++ch) {
+                    for (int ch = 0; ch < S::kVChunks * (kSplit ? 2 : 1); ++ch) {  // (chunk, term)
 #pragma unroll
                         for (int h = 0; h < NGW; h += 16) {  // 16 positions at a time
                             float o[16];
@@ -1003,7 +1043,11 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             const float4 q4 = *reinterpret_cast<const float4*>(sredq + (c0g + n) * 4);
             const float ls = (s4.x + s4.y) + (s4.z + s4.w);
             const float lq = (q4.x + q4.y) + (q4.z + q4.w);
-            inv[n] = lq > 0.f ? rcp_approx(lq) : 0.f;
+            // A split P sums to the fp32 P within 2^-17; one bf16 term is
+            // normalised by its own sum, so that a dominant token's rounding
+            // cancels between numerator and denominator.
+            const float lden = kSplit ? ls : lq;
+            inv[n] = lden > 0.f ? rcp_approx(lden) : 0.f;
             m_gt = gtg == n ? m_all[n] : m_gt;
             l_gt = gtg == n ? ls : l_gt;
         }
@@ -1030,15 +1074,28 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
             for (int ps = 0; ps < NG / L::kOutRows; ++ps) {
                 ok = wait_warp(bar0 + 8 * kOutFree, (out_it & 1) ^ 1, ctl);
                 if (!ok) break;
-                const bool f32 = !item.unsplit;
+                const bool f32 = !item.unsplit || p.out_f32;  // staged as fp32 rows
 #pragma unroll 1
                 for (int ch = 0; ch < S::kVChunks; ++ch) {
                     // positions 8ps.. hold even columns 16ps + 2i, NG/2 + 8ps.. the odd ones
+                    // (and the lo terms of a split P the same, NG further on)
                     float ev[8], od[8];
-                    const uint32_t ta = tmem + lane_base + L::kOCol + ch * NG;
+                    const uint32_t ta = tmem + lane_base + L::kOCol + ch * NP;
                     tmem_ld_x8(ta + 8 * ps, ev);
                     tmem_ld_x8(ta + NG / 2 + 8 * ps, od);
-                    tmem_ld_wait();
+                    if constexpr (kSplit) {
+                        float ev2[8], od2[8];
+                        tmem_ld_x8(ta + NG + 8 * ps, ev2);
+                        tmem_ld_x8(ta + NG + NG / 2 + 8 * ps, od2);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            ev[i] += ev2[i];
+                            od[i] += od2[i];
+                        }
+                    } else {
+                        tmem_ld_wait();
+                    }
                     const int d = ch * 128 + 32 * wq + lane;  // O^T row (lane) = output column d
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -1060,16 +1117,22 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                     if (ok) {
                         // first query column of the pass; a pass stays within one run
                         const int c0 = group_col<NG, S>(p, item.g, L::kOutRows * ps);
-                        if (f32) {
+                        if (!item.unsplit) {
                             if (item.slot >= 0)
                                 bulk_store_s2g(p.opart + ((size_t)item.slot * NG + L::kOutRows * ps) * S::kDv,
                                                smem_addr(stage_f32), L::kOutRows * S::kDv * 4);
                         } else {
                             int rows = p.N - c0;
                             rows = rows < L::kOutRows ? rows : L::kOutRows;
-                            if (rows > 0)
-                                bulk_store_s2g(p.out + ((size_t)item.b * p.N + c0) * S::kDv, smem_addr(stage_bf16),
-                                               rows * S::kDv * 2);
+                            const size_t row0 = (size_t)item.b * p.N + c0;
+                            if (rows > 0) {
+                                if (p.out_f32)
+                                    bulk_store_s2g(static_cast<float*>(p.out) + row0 * S::kDv, smem_addr(stage_f32),
+                                                   rows * S::kDv * 4);
+                                else
+                                    bulk_store_s2g(static_cast<__nv_bfloat16*>(p.out) + row0 * S::kDv,
+                                                   smem_addr(stage_bf16), rows * S::kDv * 2);
+                            }
                         }
                         bulk_commit();
                         bulk_wait_read_all();
@@ -1101,7 +1164,13 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
                         if (item.slot >= 0) p.opart[((size_t)item.slot * NG + c0g + n) * S::kDv + d] = v;
                     } else {
                         const int gc = group_col<NG, S>(p, item.g, c0g + n);
-                        if (gc < p.N) p.out[((size_t)item.b * p.N + gc) * S::kDv + d] = __float2bfloat16_rn(v);
+                        const size_t o = ((size_t)item.b * p.N + gc) * S::kDv + d;
+                        if (gc < p.N) {
+                            if (p.out_f32)
+                                static_cast<float*>(p.out)[o] = v;
+                            else
+                                static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v);
+                        }
                     }
                 }
               }
@@ -1312,12 +1381,17 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
             }
         }
     }
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 packed;
-    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(p.out + (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0) = packed;
+    const size_t o = (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0;
+    if (p.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = acc;
+    } else {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 packed;
+        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) = packed;
+    }
     if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
 }
 

@@ -19,17 +19,20 @@ namespace {
 
 using namespace mla;
 
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 constexpr int kMaxDevices = 64;
+constexpr int32_t kKnownFlags = MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL | MLA_FLAG_FP32_OUT;
 
 int validate_dims(const mla_decode_dims* d) {
     if (d == nullptr) return MLA_ERR_INVALID_ARG;
     if (d->batch < 1 || d->s_q < 1 || d->num_heads < 1 || d->num_blocks < 1 ||
         d->max_blocks_per_seq < 1 || d->num_sms < 0 || d->reserved != 0 ||
-        (d->flags & ~(MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL)) != 0 || (d->causal != 0 && d->causal != 1))
+        (d->flags & ~kKnownFlags) != 0 || (d->causal != 0 && d->causal != 1))
         return MLA_ERR_INVALID_ARG;
     if (d->page_size != kPage || d->d_qk != kDqk || d->d_v != kDv) return MLA_ERR_UNSUPPORTED;
-    if ((int64_t)d->num_heads * d->s_q > 256) return MLA_ERR_UNSUPPORTED;
+    // One or two new tokens per request (plain decode, or two-token
+    // multi-token-prediction decode with the causal rule between them).
+    if (d->s_q > 2 || (int64_t)d->num_heads * d->s_q > 256) return MLA_ERR_UNSUPPORTED;
     const Grouping gr = make_grouping(d->num_heads, d->s_q);
     const int64_t BG = (int64_t)d->batch * gr.Hg;
     // Work units and row counts must fit the int32 arithmetic of the kernels.
@@ -89,7 +92,7 @@ int validate_gqa(const mla_gqa_dims* d) {
     if (d == nullptr) return MLA_ERR_INVALID_ARG;
     if (d->batch < 1 || d->s_q < 1 || d->num_q_heads < 1 || d->num_kv_groups < 1 || d->num_blocks < 1 ||
         d->max_blocks_per_seq < 1 || d->num_sms < 0 ||
-        (d->flags & ~(MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL)) != 0 || (d->causal != 0 && d->causal != 1))
+        (d->flags & ~kKnownFlags) != 0 || (d->causal != 0 && d->causal != 1))
         return MLA_ERR_INVALID_ARG;
     if (d->page_size != kPage || d->d_head != ShapeGqa::kDh || d->d_rope != ShapeGqa::kDrope || d->s_q > 2 ||
         (int64_t)d->num_q_heads != (int64_t)kGqaHeadsPerGroup * d->num_kv_groups || d->num_kv_groups > 64)
@@ -215,12 +218,13 @@ struct ColMap {
 
 template <int kDvT>
 int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const void* workspace, void* out,
-                   float* lse, cudaStream_t stream) {
+                   float* lse, int32_t flags, cudaStream_t stream) {
     CombineParams c;
     c.sched = static_cast<const int32_t*>(schedule);
     c.opart = static_cast<const float*>(workspace);
     c.lpart = c.opart + (size_t)pl.slots * pl.gr.NG * kDvT;
-    c.out = static_cast<__nv_bfloat16*>(out);
+    c.out = out;
+    c.out_f32 = (flags & MLA_FLAG_FP32_OUT) ? 1 : 0;
     c.lse = lse;
     c.status = const_cast<int32_t*>(c.sched) + kHdrStatus;
     c.s_q = cm.s_q;
@@ -377,7 +381,8 @@ const char* mla_decode_strerror(int code) {
     switch (code) {
         case MLA_OK: return "ok";
         case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or bad dims)";
-        case MLA_ERR_UNSUPPORTED: return "unsupported shape (page_size must be 64, d_qk 576, d_v 512, heads*s_q <= 256)";
+        case MLA_ERR_UNSUPPORTED:
+            return "unsupported shape (page_size must be 64, d_qk 576, d_v 512, s_q 1 or 2, heads*s_q <= 256)";
         case MLA_ERR_CUDA: return "CUDA runtime or launch error";
         case MLA_ERR_BAD_SCHEDULE: return "schedule buffer does not match these dims";
         case MLA_ERR_SCRATCH_TOO_SMALL:
@@ -476,7 +481,8 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.block_table = block_table;
     p.seqlens = cache_seqlens;
     p.kv = static_cast<const uint8_t*>(kv_cache);
-    p.out = static_cast<__nv_bfloat16*>(out);
+    p.out = out;
+    p.out_f32 = (dims->flags & MLA_FLAG_FP32_OUT) ? 1 : 0;
     p.lse = lse;
     p.opart = static_cast<float*>(workspace);
     p.lpart = p.opart + (size_t)pl.slots * pl.gr.NG * kDv;
@@ -502,7 +508,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
                           : launch_fwd<64, ShapeMla>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
-    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, st);
+    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags, st);
 }
 
 int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const void* workspace, void* out,
@@ -512,7 +518,7 @@ int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const 
     if (rc != MLA_OK) return rc;
     if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
-    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse,
+    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags,
                                static_cast<cudaStream_t>(stream));
 }
 
@@ -562,7 +568,8 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
     p.block_table = block_table;
     p.seqlens = cache_seqlens;
     p.kv = static_cast<const uint8_t*>(kv_cache);
-    p.out = static_cast<__nv_bfloat16*>(out);
+    p.out = out;
+    p.out_f32 = (dims->flags & MLA_FLAG_FP32_OUT) ? 1 : 0;
     p.lse = lse;
     p.opart = static_cast<float*>(workspace);
     p.lpart = p.opart + (size_t)pl.slots * pl.gr.NG * ShapeGqa::kDv;
@@ -587,7 +594,7 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
     return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
-                                         pl, schedule, workspace, out, lse, st);
+                                         pl, schedule, workspace, out, lse, dims->flags, st);
 }
 
 int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,
@@ -598,7 +605,8 @@ int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const
     if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
     return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
-                                         pl, schedule, workspace, out, lse, static_cast<cudaStream_t>(stream));
+                                         pl, schedule, workspace, out, lse, dims->flags,
+                                         static_cast<cudaStream_t>(stream));
 }
 
 #ifdef MLA_TRACE

@@ -11,8 +11,12 @@ GPU shard over requests instead, with no collective at all.
 
 Page split: request b with P_b pages gives rank r the pages
 [floor(r P_b / R), floor((r + 1) P_b / R)), so the last rank always holds the
-request's last page (and so its last s_q tokens); only that rank applies the
-causal rule, every other rank's tokens are visible to all query tokens.
+request's last page.  The causal rule with s_q new tokens hides the request's
+last s_q - 1 positions from its earlier query tokens.  With s_q <= 2 that is
+at most the last position, which lies in the last page, so only the last rank
+applies the causal rule and every other rank's tokens are visible to all query
+tokens.  (With s_q >= 3 the hidden positions could straddle a rank boundary;
+the decode library takes s_q 1 or 2 only, and so does this split.)
 """
 from __future__ import annotations
 
@@ -33,8 +37,15 @@ def page_range(num_pages: int, world: int, rank: int) -> Tuple[int, int]:
     return (rank * num_pages) // world, ((rank + 1) * num_pages) // world
 
 
+def check_s_q(s_q: int) -> None:
+    """The split's causal assignment holds for one or two new tokens only."""
+    if s_q not in (1, 2):
+        raise ValueError("split-KV across ranks takes s_q 1 or 2, got %r" % (s_q,))
+
+
 def rank_causal(causal: bool, world: int, rank: int) -> bool:
-    """Whether ``rank`` applies the causal rule: only the holder of the tails."""
+    """Whether ``rank`` applies the causal rule: only the holder of the tails
+    (exact for s_q <= 2, see the module docstring)."""
     return bool(causal) and rank == world - 1
 
 
@@ -80,6 +91,7 @@ class KvSplitDecoder:
 
     def __init__(self, batch: int, s_q: int, num_heads: int, num_blocks: int, max_blocks_per_seq: int,
                  causal: bool = False, group=None, device: Optional[torch.device] = None):
+        check_s_q(s_q)
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -109,6 +121,7 @@ class KvSplitGqaDecoder:
 
     def __init__(self, batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
                  causal: bool = False, group=None, device: Optional[torch.device] = None):
+        check_s_q(s_q)
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)

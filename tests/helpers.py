@@ -34,9 +34,11 @@ def bf16_floor(ref: np.ndarray) -> float:
 
 def compare(out_gpu: torch.Tensor, lse_gpu: torch.Tensor, ref_out: np.ndarray, ref_lse: np.ndarray,
             rows=None, heads=None, s_q=None):
-    """out_gpu [B,s_q,h,512] bf16, lse_gpu [B,h,s_q] fp32 (device or host);
+    """out_gpu [B,s_q,h,512] bf16 (or fp32), lse_gpu [B,h,s_q] fp32 (device or host);
     ref_* from the oracle over flattened rows r = (b*s_q+s)*h+head (all, or ``rows``).
-    Returns a dict of metrics and asserts the tolerances."""
+    Returns a dict of metrics and asserts the tolerances.  An fp32 output (the
+    result before any bf16 rounding) is held to the literal RMSE bar, with no
+    allowance for the bf16 rounding floor."""
     B, sq, h, dv = out_gpu.shape
     o = out_gpu.detach().double().cpu().numpy().reshape(B * sq * h, dv)
     l = lse_gpu.detach().double().cpu().numpy()  # [B, h, s_q]
@@ -54,7 +56,8 @@ def compare(out_gpu: torch.Tensor, lse_gpu: torch.Tensor, ref_out: np.ndarray, r
     )
     lse_err = np.abs(l[finite] - ref_lse[finite]) / np.maximum(1.0, np.abs(ref_lse[finite]))
     m["lse_rel_err"] = float(lse_err.max()) if lse_err.size else 0.0
-    m["rmse_bar"] = RMSE_BAR if m["q_floor"] <= 2.5e-4 else RMSE_BAR + m["q_floor"]
+    literal = out_gpu.dtype == torch.float32 or m["q_floor"] <= 2.5e-4
+    m["rmse_bar"] = RMSE_BAR if literal else RMSE_BAR + m["q_floor"]
     assert np.isfinite(o).all(), "non-finite output"
     assert np.array_equal(np.isneginf(l), np.isneginf(ref_lse)), "LSE -inf pattern differs"
     assert not np.isnan(l).any()

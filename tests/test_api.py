@@ -43,7 +43,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_version_and_strerror(lib):
-    assert bd.mla_decode_version() == 4
+    assert bd.mla_decode_version() == 5
     for code in (0, -1, -2, -3, -4):
         assert bd.mla_decode_strerror(code)
     assert "unknown" in bd.mla_decode_strerror(-99)
@@ -65,7 +65,7 @@ def test_sizes_need_valid_dims(lib):
     wide = _dims(s_q=2, num_heads=128, batch=32)  # 256 columns -> 4 groups of 64
     assert bd.mla_decode_schedule_bytes(wide) == 4 * (16 + 8 * 148 + 3 * 32 * 4 + 1)
     assert bd.mla_decode_workspace_bytes(wide) == 2 * 148 * 64 * 513 * 4
-    for bad in (dict(batch=0), dict(s_q=0), dict(num_heads=0), dict(num_blocks=0),
+    for bad in (dict(batch=0), dict(s_q=0), dict(s_q=3), dict(num_heads=0), dict(num_blocks=0),
                 dict(max_blocks_per_seq=0), dict(num_sms=-1)):
         assert bd.mla_decode_schedule_bytes(_dims(**bad)) == 0, bad
         assert bd.mla_decode_workspace_bytes(_dims(**bad)) == 0, bad
@@ -86,6 +86,8 @@ def test_fwd_rejects_bad_dims_before_any_launch(lib):
         (dict(d_qk=512), bd.MLA_ERR_UNSUPPORTED),
         (dict(d_v=576), bd.MLA_ERR_UNSUPPORTED),
         (dict(num_heads=129, s_q=2), bd.MLA_ERR_UNSUPPORTED),
+        (dict(s_q=3), bd.MLA_ERR_UNSUPPORTED),
+        (dict(s_q=4, num_heads=2), bd.MLA_ERR_UNSUPPORTED),
         (dict(batch=0), bd.MLA_ERR_INVALID_ARG),
         (dict(causal=2), bd.MLA_ERR_INVALID_ARG),
         (dict(reserved=1), bd.MLA_ERR_INVALID_ARG),

@@ -53,6 +53,21 @@ def test_shard_reassembles_the_batch():
     assert not kv_split.rank_causal(False, 3, 2)
 
 
+def test_split_takes_one_or_two_new_tokens():
+    """With s_q = 3 the two hidden positions of query token 0 can straddle a
+    rank boundary (L = 65 over 2 ranks: rank 0 holds position 63), so the split
+    refuses it, as the decode library does."""
+    kv_split.check_s_q(1)
+    kv_split.check_s_q(2)
+    for bad in (0, 3, 4):
+        with pytest.raises(ValueError):
+            kv_split.check_s_q(bad)
+        with pytest.raises(ValueError):
+            kv_split.KvSplitDecoder(1, bad, 16, 10, 10, causal=True)
+        with pytest.raises(ValueError):
+            kv_split.KvSplitGqaDecoder(1, bad, 1, 10, 10, causal=True)
+
+
 def _shard_oracle(d, R, causal):
     outs, lses = [], []
     for r in range(R):
