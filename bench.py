@@ -51,6 +51,8 @@ def parse_args():
                     help="decode only the first BATCH requests of the workload (small profiling case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cases", action="store_true",
+                    help="leave out the per-workload cases (every named workload: timing and all-rows parity)")
     ap.add_argument("--gqa", action="store_true",
                     help="GQA path over a group-expanded cache (bs16, s_q 2 causal, 8 KV groups = 128 query "
                          "heads, 16K context): one JSON line")
@@ -262,28 +264,34 @@ def oracle_sample_rate(d, w, budget_s: float, max_requests=None, collect=None):
     return done_bytes / elapsed / 1e9, elapsed, sample, cores
 
 
-def bench_parity(done, out_rows, lse_rows):
-    """Outputs of the timed launch configuration against the oracle rows the
-    CPU baseline computed: max|err| relative to max|ref|, RMSE (with the
-    bf16 rounding floor of the exact result), LSE relative error."""
+def parity_metrics(ref, ref_l, got, got_l):
+    """max|err| relative to max|ref|, RMSE (with the bf16 rounding floor of
+    the exact result), LSE relative error of ``got`` rows against the fp64
+    oracle's ``ref`` rows."""
     import numpy as np
-    if not done:
-        return None
-    rows = np.concatenate([np.asarray(r) for r, _, _ in done])
-    ref = np.concatenate([o for _, o, _ in done])
-    ref_l = np.concatenate([l for _, _, l in done])
-    got = out_rows[rows].astype(np.float64)
-    got_l = lse_rows[rows].astype(np.float64)
-    err = got - ref
+    err = got.astype(np.float64) - ref
+    got_l = got_l.astype(np.float64)
     bf = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
     fin = np.isfinite(ref_l)
-    return {"rows": int(rows.size), "oracle": "fp64",
+    return {"rows": int(ref.shape[0]), "oracle": "fp64",
             "max_abs_err_over_max_ref": float(np.abs(err).max() / max(np.abs(ref).max(), 1e-30)),
             "rmse": float(np.sqrt(np.mean(err ** 2))),
             "bf16_floor_rmse": float(np.sqrt(np.mean((bf - ref) ** 2))),
             "lse_rel_err": float((np.abs(got_l[fin] - ref_l[fin]) / np.maximum(1.0, np.abs(ref_l[fin]))).max())
             if fin.any() else 0.0,
             "lse_neginf_match": bool(np.array_equal(np.isneginf(got_l), np.isneginf(ref_l)))}
+
+
+def bench_parity(done, out_rows, lse_rows):
+    """Outputs of the timed launch configuration against the oracle rows the
+    CPU baseline computed."""
+    import numpy as np
+    if not done:
+        return None
+    rows = np.concatenate([np.asarray(r) for r, _, _ in done])
+    ref = np.concatenate([o for _, o, _ in done])
+    ref_l = np.concatenate([l for _, _, l in done])
+    return parity_metrics(ref, ref_l, out_rows[rows], lse_rows[rows])
 
 
 def run_reference(args, w):
@@ -459,6 +467,8 @@ def run_ours(args, w):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world)
+    del q, kv, bt, sl, sched, ws, out, lse, flush
+    torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:
@@ -478,6 +488,9 @@ def run_ours(args, w):
         cpu = {"value": r, "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": sample + " (%.1f s)" % t}
         parity = bench_parity(done, out_check, lse_check)
+    cases = None
+    if world == 1 and not args.no_cases:
+        cases = run_cases(args, dev, w, d, hbm_peak, tf_peak)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": ms_step * 1e3,
@@ -495,6 +508,7 @@ def run_ours(args, w):
         "e2e": e2e,
         "clocks": clocks.summary(wall0, wall1),
         "gpu_launches": 3 * args.steps,
+        "cases": cases,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -582,6 +596,122 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
             "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": res_bytes,
             "note": "q, block_table, cache_seqlens uploaded (one packed copy) and out, lse read back (one packed "
                     "copy) every step, inside one CUDA-graph replay per step, then a stream sync; KV cache resident"}
+
+
+def measure_case(w, d, dev, steps, warmup, hbm_peak, tf_peak):
+    """One named workload on this GPU: the step (schedule + decode + combine)
+    and the decode kernel alone, each graph-replayed with CUDA events around
+    every replay (L2 flushed before each replay, untimed, where the KV fits
+    twice into L2); median and best per call.  Then one more step in bf16 and
+    one with MLA_FLAG_FP32_OUT, both checked against the fp64 oracle on every
+    row of the workload."""
+    import numpy as np
+    import oracle
+    stream = torch.cuda.current_stream(dev)
+    q = d["q"].to(dev)
+    kv = d["kv_cache"].to(dev)
+    bt = d["block_table"].to(dev)
+    sl = d["cache_seqlens"].to(dev)
+    B, s_q, h = w.batch, w.s_q, w.heads
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mk = lambda flags=0: bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms, flags)
+    dims, dims_nc, dims_f32 = mk(), mk(bd.MLA_FLAG_NO_COMBINE), mk(bd.MLA_FLAG_FP32_OUT)
+    sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
+    ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, s_q, h, 512, dtype=torch.bfloat16, device=dev)
+    out32 = torch.empty(B, s_q, h, 512, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, h, s_q, dtype=torch.float32, device=dev)
+    byt = algorithmic_bytes(d["cache_seqlens"], s_q, h)
+    flops = algorithmic_flops(d["cache_seqlens"], s_q, h)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if byt["kv"] <= 2 * 126e6 else None
+    scale = d["softmax_scale"]
+
+    graphs = []
+    for dm in (dims, dims_nc):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            bd.mla_decode_get_schedule(dims, sl, sched, cap)
+            bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, scale, out, lse, cap)
+            with torch.cuda.graph(g, stream=cap):
+                if dm is dims:
+                    bd.mla_decode_get_schedule(dims, sl, sched, cap)
+                bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, scale, out, lse, cap)
+        stream.wait_stream(cap)
+        graphs.append(g)
+    times = []
+    for g in graphs:
+        ev = []
+        for i in range(max(3, warmup) + steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            if i >= max(3, warmup):
+                ev.append((a, b))
+        torch.cuda.synchronize()
+        times.append(sorted(x.elapsed_time(y) for x, y in ev))
+    del graphs
+    status = bd.mla_decode_get_status(sched)
+    (step_ms, kern_ms) = times
+    med = lambda t: statistics.median(t)
+
+    # parity, every row: the bf16 output and the fp32 output before the cast
+    bd.mla_decode_get_schedule(dims, sl, sched, stream)
+    bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, scale, out, lse, stream)
+    torch.cuda.synchronize()
+    o16 = out.float().cpu().numpy().reshape(-1, 512)
+    l16 = lse.cpu().numpy().transpose(0, 2, 1).reshape(-1)
+    bd.mla_decode_fwd(dims_f32, sched, ws, q, kv, bt, sl, scale, out32, lse, stream)
+    torch.cuda.synchronize()
+    status |= bd.mla_decode_get_status(sched)
+    o32 = out32.cpu().numpy().reshape(-1, 512)
+    l32 = lse.cpu().numpy().transpose(0, 2, 1).reshape(-1)
+    del q, kv, bt, sl, sched, ws, out, out32, lse, flush
+    torch.cuda.empty_cache()
+    t0 = time.perf_counter()
+    ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"], scale,
+                                   causal=d["causal"])
+    t_oracle = time.perf_counter() - t0
+    par = parity_metrics(ro, rl, o16, l16)
+    par["fp32_output"] = parity_metrics(ro, rl, o32, l32)
+    par["note"] = ("every row; fp32_output is MLA_FLAG_FP32_OUT, the result before the bf16 cast, held to the "
+                   "literal RMSE 5e-4")
+    t_hbm = byt["total"] / (hbm_peak * 1e9)
+    t_tc = flops / (tf_peak * 1e12)
+    roof_s = max(t_hbm, t_tc)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    return {
+        "workload": w.name, "description": w.description, "batch": B, "s_q": s_q, "heads": h,
+        "kv_tokens": kv_tokens(d["cache_seqlens"]), "kv_bytes": byt["kv"], "algorithmic_bytes": byt["total"],
+        "flops": flops,
+        "us_per_call": {"median": 1e3 * med(step_ms), "best": 1e3 * step_ms[0]},
+        "kernel_us": {"median": 1e3 * med(kern_ms), "best": 1e3 * kern_ms[0]},
+        "kv_gbs": byt["kv"] / (med(step_ms) * 1e-3) / 1e9,
+        "tflops": flops / (med(step_ms) * 1e-3) / 1e12,
+        "roofline": {"bound": bound, "us": roof_s * 1e6,
+                     "frac_step": roof_s / (med(step_ms) * 1e-3), "frac_kernel": roof_s / (med(kern_ms) * 1e-3),
+                     "kernel_achieved": (byt["total"] / (med(kern_ms) * 1e-3) / 1e9) if bound == "hbm"
+                     else flops / (med(kern_ms) * 1e-3) / 1e12,
+                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                     "peak": hbm_peak if bound == "hbm" else tf_peak},
+        "l2": "flushed before every replay (untimed)" if byt["kv"] <= 2 * 126e6 else "inputs larger than L2: no flush",
+        "steps": steps, "parity": par, "oracle_s": t_oracle, "status": status,
+    }
+
+
+def run_cases(args, dev, main_w, main_d, hbm_peak, tf_peak):
+    """Every named workload (the main one with the inputs already drawn)."""
+    cases = []
+    for name, w in workloads.WORKLOADS.items():
+        d = main_d if name == main_w.name and main_w.batch == w.batch else workloads.make_inputs(w)
+        cases.append(measure_case(w, d, dev, args.steps, args.warmup, hbm_peak, tf_peak))
+        del d
+    return cases
 
 
 SWEEP_BATCH = (1, 4, 8, 16, 32)

@@ -284,8 +284,9 @@ int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, v
  * Split-KV across GPUs: merge of per-rank decode results.  Each of R ranks
  * decodes the same queries against a disjoint part of every request's KV
  * (for example a contiguous range of its pages, held in that rank's own
- * pool); the ranks exchange their bf16 outputs and fp32 LSEs (an all-gather
- * over NVLink) and each merges them with this call:
+ * pool); the ranks exchange their outputs and fp32 LSEs (an all-gather over
+ * NVLink) and each merges them with this call (bf16 outputs) or with
+ * mla_decode_combine_ranks_f32 (fp32 outputs):
  *
  *   L* = log sum_i exp(lse_i),  out = sum_i exp(lse_i - L*) o_i,  lse = L*
  *
@@ -312,6 +313,16 @@ int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, v
 int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
                              const void* o_parts, const float* lse_parts, void* out, float* lse,
                              void* stream);
+
+/* The same merge of fp32 per-rank results: o_parts fp32 [num_ranks][batch]
+ * [s_q][num_heads][d_v], as mla_decode_fwd / mla_gqa_decode_fwd write them
+ * with MLA_FLAG_FP32_OUT.  The merged row is rounded to bf16 once, as the
+ * combine of split partials inside one GPU does; exchanging bf16 outputs
+ * instead rounds each rank's result first.  Other arguments and errors as
+ * for mla_decode_combine_ranks. */
+int mla_decode_combine_ranks_f32(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads,
+                                 int32_t d_v, const float* o_parts, const float* lse_parts, void* out,
+                                 float* lse, void* stream);
 
 /* Library ABI version (increments on any change of these declarations). */
 int mla_decode_version(void);

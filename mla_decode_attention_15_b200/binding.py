@@ -56,6 +56,7 @@ EXPORTED = (
     "mla_absorb_q",
     "mla_absorb_o",
     "mla_decode_combine_ranks",
+    "mla_decode_combine_ranks_f32",
 )
 
 GQA_D_HEAD = 128
@@ -140,8 +141,9 @@ def lib() -> ctypes.CDLL:
         L.mla_gqa_decode_combine.restype = ctypes.c_int
         L.mla_gqa_decode_combine.argtypes = [Q, vp, vp, vp, vp, vp]
         i32 = ctypes.c_int32
-        L.mla_decode_combine_ranks.restype = ctypes.c_int
-        L.mla_decode_combine_ranks.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+        for name in ("mla_decode_combine_ranks", "mla_decode_combine_ranks_f32"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         A = ctypes.POINTER(mla_absorb_dims)
         for name in ("mla_absorb_q", "mla_absorb_o"):
             getattr(L, name).restype = ctypes.c_int
@@ -347,11 +349,13 @@ class GqaDecoder:
     MlaDecoder."""
 
     def __init__(self, batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
-                 causal: bool = False, num_sms: int = 0, device: Optional[torch.device] = None):
+                 causal: bool = False, num_sms: int = 0, device: Optional[torch.device] = None,
+                 fp32_out: bool = False):
         self.device = torch.device(device or "cuda")
         if num_sms == 0:
             num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
-        self.dims = make_gqa_dims(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq, causal, num_sms)
+        self.dims = make_gqa_dims(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq, causal, num_sms,
+                                  MLA_FLAG_FP32_OUT if fp32_out else 0)
         sb = mla_gqa_decode_schedule_bytes(self.dims)
         wb = mla_gqa_decode_workspace_bytes(self.dims)
         if sb == 0 or wb == 0:
@@ -360,7 +364,8 @@ class GqaDecoder:
         self.row_width = 2 * num_kv_groups * GQA_D_HEAD + GQA_D_ROPE
         self.schedule = torch.empty(sb, dtype=torch.uint8, device=self.device)
         self.workspace = torch.empty(wb, dtype=torch.uint8, device=self.device)
-        self.out = torch.empty(batch, s_q, h, GQA_D_HEAD, dtype=torch.bfloat16, device=self.device)
+        self.out = torch.empty(batch, s_q, h, GQA_D_HEAD, dtype=torch.float32 if fp32_out else torch.bfloat16,
+                               device=self.device)
         self.lse = torch.empty(batch, h, s_q, dtype=torch.float32, device=self.device)
 
     def check_inputs(self, q, kv_cache, block_table, cache_seqlens) -> None:
@@ -456,11 +461,12 @@ def absorb_o(o: torch.Tensor, w_uv: torch.Tensor, out: Optional[torch.Tensor] = 
 # ---------------------------------------------------------------- split-KV across ranks
 def mla_decode_combine_ranks(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor,
                              lse: torch.Tensor, stream=None) -> None:
-    """o_parts bf16 [R, B, s_q, h, d_v], lse_parts fp32 [R, B, h, s_q] -> out
-    bf16 [B, s_q, h, d_v], lse fp32 [B, h, s_q]: the LSE-weighted merge of the
-    ranks' results (d_v 512 or 128)."""
-    _require(o_parts.dim() == 5 and o_parts.dtype == torch.bfloat16 and o_parts.is_contiguous(),
-             "o_parts must be contiguous bf16 [R, B, s_q, h, d_v]")
+    """o_parts bf16 or fp32 [R, B, s_q, h, d_v], lse_parts fp32 [R, B, h, s_q]
+    -> out bf16 [B, s_q, h, d_v], lse fp32 [B, h, s_q]: the LSE-weighted merge
+    of the ranks' results (d_v 512 or 128); fp32 parts are rounded once, after
+    the merge."""
+    _require(o_parts.dim() == 5 and o_parts.dtype in (torch.bfloat16, torch.float32) and o_parts.is_contiguous(),
+             "o_parts must be contiguous bf16 or fp32 [R, B, s_q, h, d_v]")
     R, B, s_q, h, d_v = o_parts.shape
     _require(lse_parts.dtype == torch.float32 and lse_parts.is_contiguous() and
              tuple(lse_parts.shape) == (R, B, h, s_q), "lse_parts must be contiguous fp32 [R, B, h, s_q]")
@@ -470,9 +476,9 @@ def mla_decode_combine_ranks(o_parts: torch.Tensor, lse_parts: torch.Tensor, out
              "lse must be contiguous fp32 [B, h, s_q]")
     for t in (lse_parts, out, lse):
         _require(t.device == o_parts.device, "all tensors must be on %s" % o_parts.device)
-    _check(lib().mla_decode_combine_ranks(int(R), int(B), int(s_q), int(h), int(d_v), _ptr(o_parts),
-                                          _ptr(lse_parts), _ptr(out), _ptr(lse), _stream(stream)),
-           "mla_decode_combine_ranks")
+    fn = lib().mla_decode_combine_ranks_f32 if o_parts.dtype == torch.float32 else lib().mla_decode_combine_ranks
+    _check(fn(int(R), int(B), int(s_q), int(h), int(d_v), _ptr(o_parts), _ptr(lse_parts), _ptr(out), _ptr(lse),
+              _stream(stream)), "mla_decode_combine_ranks")
 
 
 def absorbed_mla_decode(q_in: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor, kv_cache: torch.Tensor,

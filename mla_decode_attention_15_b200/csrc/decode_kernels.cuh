@@ -608,7 +608,7 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
     it.init(meta);
     Item item;
     uint32_t s_it = 0, q_it = 0;
-    bool ok = true, issued = false;
+    bool ok = true;
 #ifdef MLA_TRACE
     Tracer tracer_(issuer == 0 ? 1 : 0, issuer == 0);
 #endif
@@ -642,7 +642,6 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
                     first = false;
                 }
             }
-            issued = true;
             umma_commit(bar0 + 8 * (kSFull0 + sb));
             MLA_TRACE_EV(kTrMmaG1Issued);
             if (j == item.p1 - 1) umma_commit(bar0 + 8 * kQEmpty);
@@ -650,10 +649,11 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
         }
         ++q_it;
     }
-    if (issued) {
-        umma_commit(bar0 + 8 * kMmaDone);
-        wait_drain(bar0 + 8 * kMmaDone, 0);
-    }
+    // Drain before TMEM is released, on the normal and the abort path alike:
+    // every GEMM1 issuer commits (a commit with no MMA outstanding arrives at
+    // once), so the barrier completes as soon as all their MMAs are done.
+    umma_commit(bar0 + 8 * kMmaDone);
+    wait_drain(bar0 + 8 * kMmaDone, 0);
 }
 
 // GEMM2 issuer: O^T[512 x NG] += V^T[512 x 64] . P^T as soon as P^T is in
@@ -677,7 +677,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
     it.init(meta);
     Item item;
     uint32_t s_it = 0, item_it = 0;
-    bool ok = true, issued = false;
+    bool ok = true;
 #ifdef MLA_TRACE
     Tracer tracer_(issuer == 0 ? 2 : 0, issuer == 0);
 #endif
@@ -708,7 +708,6 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
                     umma_f16(tmem + L::kOCol + ch * NP, a, b, kIdescO, (first && k == 0) ? 0u : 1u);
                 }
             }
-            issued = true;
             umma_commit(bar0 + 8 * (kKvEmpty0 + st));
             umma_commit(bar0 + 8 * (kPEmpty0 + pb));
             MLA_TRACE_EV(kTrMmaG2Issued);
@@ -717,10 +716,9 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
         if (!ok) break;
         ++item_it;
     }
-    if (issued) {
-        umma_commit(bar0 + 8 * kMmaDone2);
-        wait_drain(bar0 + 8 * kMmaDone2, 0);
-    }
+    // drained as GEMM1's issuers are
+    umma_commit(bar0 + 8 * kMmaDone2);
+    wait_drain(bar0 + 8 * kMmaDone2, 0);
 }
 
 template <int NG, class S>

@@ -675,8 +675,13 @@ int mla_absorb_o(const mla_absorb_dims* dims, const void* o, const void* w_uv, v
     return launch_absorb<1>(dims, o, w_uv, out, status, static_cast<cudaStream_t>(stream));
 }
 
-int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
-                             const void* o_parts, const float* lse_parts, void* out, float* lse, void* stream) {
+}  // extern "C"
+
+namespace {
+
+template <typename TIn>
+int combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
+                  const void* o_parts, const float* lse_parts, void* out, float* lse, void* stream) {
     if (num_ranks < 1 || num_ranks > kRankCombineMaxRanks || batch < 1 || s_q < 1 || num_heads < 1)
         return MLA_ERR_INVALID_ARG;
     if (d_v != kDv && d_v != ShapeGqa::kDv) return MLA_ERR_UNSUPPORTED;
@@ -686,7 +691,7 @@ int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int3
     if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
     RankCombineParams p;
-    p.o_parts = static_cast<const __nv_bfloat16*>(o_parts);
+    p.o_parts = o_parts;
     p.lse_parts = lse_parts;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
@@ -696,10 +701,25 @@ int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int3
     p.h = num_heads;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d_v == kDv)
-        mla_rank_combine_kernel<kDv><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
+        mla_rank_combine_kernel<kDv, TIn><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
     else
-        mla_rank_combine_kernel<ShapeGqa::kDv><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
+        mla_rank_combine_kernel<ShapeGqa::kDv, TIn><<<(unsigned)blocks, 32 * kRankCombineWarps, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_combine_ranks(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
+                             const void* o_parts, const float* lse_parts, void* out, float* lse, void* stream) {
+    return combine_ranks<__nv_bfloat16>(num_ranks, batch, s_q, num_heads, d_v, o_parts, lse_parts, out, lse, stream);
+}
+
+int mla_decode_combine_ranks_f32(int32_t num_ranks, int32_t batch, int32_t s_q, int32_t num_heads, int32_t d_v,
+                                 const float* o_parts, const float* lse_parts, void* out, float* lse,
+                                 void* stream) {
+    return combine_ranks<float>(num_ranks, batch, s_q, num_heads, d_v, o_parts, lse_parts, out, lse, stream);
 }
 
 }  // extern "C"

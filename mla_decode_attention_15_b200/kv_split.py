@@ -2,10 +2,11 @@
 
 Each of R ranks holds a contiguous part of every request's KV pages in its own
 pool and decodes the same queries against it with the single-GPU path; the
-ranks then exchange their results (bf16 O and fp32 LSE, one all-gather each,
-over NVLink with NCCL) and every rank merges them with
-``mla_decode_combine_ranks``: L* = log sum_i exp(lse_i), O = sum_i
-exp(lse_i - L*) O_i.  That exchange is the one collective the path needs when
+ranks then exchange their results (fp32 O before any bf16 rounding, and fp32
+LSE; one all-gather each, over NVLink with NCCL) and every rank merges them
+with ``mla_decode_combine_ranks_f32``: L* = log sum_i exp(lse_i), O = sum_i
+exp(lse_i - L*) O_i, rounded to bf16 once, as the combine of split partials
+inside one GPU does.  That exchange is the one collective the path needs when
 a single request's context is spread over several GPUs; batches that fit one
 GPU shard over requests instead, with no collective at all.
 
@@ -85,7 +86,7 @@ def gather(local: torch.Tensor, group=None) -> torch.Tensor:
 
 class KvSplitDecoder:
     """One rank's part of an MLA decode whose KV is split across the ranks of
-    ``group``: local decode, all-gather of (O, LSE), merge.  Shapes as for
+    ``group``: local decode (fp32 output), all-gather of (O, LSE), merge.  Shapes as for
     ``MlaDecoder``; ``num_blocks`` / ``max_blocks_per_seq`` describe this
     rank's pool and local block table."""
 
@@ -96,7 +97,7 @@ class KvSplitDecoder:
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.dec = bd.MlaDecoder(batch, s_q, num_heads, num_blocks, max_blocks_per_seq,
-                                 rank_causal(causal, self.world, self.rank), device=device)
+                                 rank_causal(causal, self.world, self.rank), device=device, fp32_out=True)
         dev = self.dec.device
         self.out = torch.empty(batch, s_q, num_heads, bd.D_V, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(batch, num_heads, s_q, dtype=torch.float32, device=dev)
@@ -126,7 +127,7 @@ class KvSplitGqaDecoder:
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.dec = bd.GqaDecoder(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq,
-                                 rank_causal(causal, self.world, self.rank), device=device)
+                                 rank_causal(causal, self.world, self.rank), device=device, fp32_out=True)
         dev = self.dec.device
         h = self.dec.dims.num_q_heads
         self.out = torch.empty(batch, s_q, h, bd.GQA_D_HEAD, dtype=torch.bfloat16, device=dev)
