@@ -190,6 +190,9 @@ enum TraceTag : unsigned {
     kTrSmEpiLse = 14,   // softmax: LSE written (epilogue)
     kTrMmaG1Issued = 15,  // gemm1 issuer: MMAs issued and committed
     kTrMmaG2Issued = 16,  // gemm2 issuer: MMAs issued and committed
+    kTrBoxIssued = 17,    // CTA-pair producer: one GEMM1 box load issued
+    kTrBoxFull = 18,      // CTA-pair issuer: one GEMM1 box seen full
+    kTrBoxEmpty = 19,     // CTA-pair producer: one GEMM1 slot seen empty
 };
 struct Tracer {
     int cta, role;
@@ -253,9 +256,14 @@ struct CombineParams {
     void* out;  // bf16 rows, or fp32 rows when out_f32
     float* lse;
     int32_t* status;
-    int s_q, heads, N, NG, Hg, G, BG, slots_cap;
+    int s_q, heads, N, NG, Hg, G, BG, slots_cap;  // Hg, BG: head groups per request, request-groups
     int run_rows, run_stride;
     int out_f32;
+    // The plan's own shape: plan_BG work items per plan row of bginfo, and
+    // share = head groups that walked each work range side by side (1: the
+    // plan has one row per request-group; else one row per request, and split
+    // i of group g sits in slot (base + i) * share + g).
+    int plan_BG, plan_Hg, shift, share;
 };
 
 // ------------------------------------------------------------------ layout
@@ -1202,7 +1210,8 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
     griddep_launch_dependents();
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
-        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG) {
+        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG ||
+        __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != 1) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
@@ -1310,7 +1319,8 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     // start only after its own wait on the grid that wrote the plan.
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
-        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != p.NG) {
+        __ldg(hdr + kHdrBG) != p.plan_BG || __ldg(hdr + kHdrHg) != p.plan_Hg || __ldg(hdr + kHdrNG) != p.NG ||
+        __ldg(hdr + kHdrShift) != p.shift || __ldg(hdr + kHdrShareHg) != p.share) {
         if (threadIdx.x == 0 && bg == 0 && n == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
@@ -1319,20 +1329,24 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     // one run (MLA groups): no division
     const int gc = p.run_stride == 0 ? g * p.run_rows + n : item_col(p.run_rows, p.run_stride, g, n);
     if (gc >= p.N) return;
-    const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * bg;
+    const int row = p.share > 1 ? b : bg;  // plan row of this request-group
+    const int gs = p.share > 1 ? g : 0;
+    const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * row;
     const int base = __ldg(info + 0);
     const int k = __ldg(info + 1);
     if (k == 1) return;  // unsplit: the decode kernel wrote the final row
-    if (k > 1 && (base < 0 || base + k > p.slots_cap)) {
+    if (k > 1 && (base < 0 || ((int64_t)base + k) * p.share > p.slots_cap)) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
     const int s = gc / p.heads;
     const int head = gc - s * p.heads;
     const int d0 = threadIdx.x * 4;
-    const float* lp = p.lpart + (size_t)base * p.NG + n;
-    const float* op = p.opart + ((size_t)base * p.NG + n) * kDv + d0;
-    const size_t ostride = (size_t)p.NG * kDv;
+    const size_t slot0 = (size_t)base * p.share + gs;
+    const size_t lstride = (size_t)p.share * p.NG;  // split i -> slot0 + i * share
+    const float* lp = p.lpart + slot0 * p.NG + n;
+    const float* op = p.opart + (slot0 * p.NG + n) * kDv + d0;
+    const size_t ostride = lstride * kDv;
     griddep_wait();  // the decode grid's partials are complete and visible
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lstar = -INFINITY;
@@ -1341,15 +1355,15 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
 #pragma unroll
         for (int i = 0; i < kCombinePre; ++i)
             if (i < k) pre[i] = __ldg(reinterpret_cast<const float4*>(op + (size_t)i * ostride));
-        float own = threadIdx.x < k ? __ldg(lp + (size_t)threadIdx.x * p.NG) : -INFINITY;
+        float own = threadIdx.x < k ? __ldg(lp + (size_t)threadIdx.x * lstride) : -INFINITY;
         float mx = own;
         for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads)
-            mx = fmaxf(mx, __ldg(lp + (size_t)i * p.NG));
+            mx = fmaxf(mx, __ldg(lp + (size_t)i * lstride));
         mx = combine_block_reduce<kCombineThreads, true>(mx, red);
         if (mx != -INFINITY) {  // uniform across the block
             float sum = 0.f;
             for (int i = threadIdx.x; i < k; i += kCombineThreads)
-                sum += expf((i == threadIdx.x ? own : __ldg(lp + (size_t)i * p.NG)) - mx);
+                sum += expf((i == threadIdx.x ? own : __ldg(lp + (size_t)i * lstride)) - mx);
             sum = combine_block_reduce<kCombineThreads, false>(sum, red);
             lstar = mx + logf(sum);
             for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
@@ -1357,7 +1371,7 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
                 __syncthreads();  // the previous chunk's weights are consumed
                 if (threadIdx.x < cn)
                     wts[threadIdx.x] =
-                        expf((c0 == 0 ? own : __ldg(lp + (size_t)(c0 + threadIdx.x) * p.NG)) - lstar);
+                        expf((c0 == 0 ? own : __ldg(lp + (size_t)(c0 + threadIdx.x) * lstride)) - lstar);
                 __syncthreads();
                 int i = 0;
                 if (c0 == 0) {
@@ -1424,7 +1438,7 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
 // prefix is also written to the schedule buffer.
 __global__ void __launch_bounds__(1024)
     mla_decode_schedule_kernel(const int32_t* __restrict__ seqlens_g, int32_t* __restrict__ sched, int B,
-                               int Hg, int NG, int G, int max_blocks, int use_smem) {
+                               int Hg, int NG, int G, int max_blocks, int use_smem, int shift, int share_hg) {
     extern __shared__ int32_t sh[];
     __shared__ int warp_tot[32];
     __shared__ int carry;
@@ -1454,7 +1468,7 @@ __global__ void __launch_bounds__(1024)
         if (bg < BG) {
             const int L = seqlens[bg / Hg];
             if (!seqlen_in_range(L, max_blocks)) bad_len = 1;
-            v = (int)units_of(pages_of(clamp_seqlen(L, max_blocks)));
+            v = (int)units_of(blocks_of(clamp_seqlen(L, max_blocks), shift));
         }
         const int incl = block_inclusive_scan(v, warp_tot);
         if (bg < BG) {
@@ -1473,14 +1487,14 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
     const int64_t T = units_per_cta(W, G);
     for (int k = threadIdx.x; k < G; k += 1024)
-        cta_meta(prefix, BG, W, T, k, seqlens, Hg, max_blocks, meta + (size_t)k * kMetaWords);
+        cta_meta(prefix, BG, W, T, k, seqlens, Hg, max_blocks, shift, meta + (size_t)k * kMetaWords);
     __syncthreads();
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     for (int base = 0; base < BG; base += 1024) {
         const int bg = base + threadIdx.x;
         int ns = 0;
-        if (bg < BG) ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, max_blocks), T);
+        if (bg < BG) ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, max_blocks, shift), T);
         const int v = ns > 1 ? ns : 0;
         const int incl = block_inclusive_scan(v, warp_tot);
         if (bg < BG) {
@@ -1503,7 +1517,9 @@ __global__ void __launch_bounds__(1024)
         sched[kHdrW] = (int)W;
         sched[kHdrBatch] = B;
         sched[kHdrMaxBlocks] = max_blocks;
-        for (int i = kHdrMaxBlocks + 1; i < kHdrWords; ++i) sched[i] = 0;
+        sched[kHdrShift] = shift;
+        sched[kHdrShareHg] = share_hg;
+        for (int i = kHdrShareHg + 1; i < kHdrWords; ++i) sched[i] = 0;
     }
 }
 

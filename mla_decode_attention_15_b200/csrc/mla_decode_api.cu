@@ -11,6 +11,7 @@
 
 #include "absorb_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "pair_kernels.cuh"
 #include "rank_combine.cuh"
 #include "mla_decode.h"
 #include "schedule.cuh"
@@ -62,21 +63,80 @@ int resolve_ctas(const mla_decode_dims* d, int* G) {
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A launch plan.  G and BG are the split-KV plan's own shape: work ranges
+// and plan rows (request-groups for the one-CTA kernels; requests for the
+// CTA-pair kernel, whose ranges are walked by all head groups side by side).
 struct Plan {
     Grouping gr;
-    int G;
-    int BG;
+    int G;        // work ranges of the plan
+    int BG;       // plan rows
+    int plan_Hg;  // head groups per plan row (1 for the pair kernel's plan)
+    int shift;    // log2 tokens per plan unit
+    int share;    // head groups walking each range (1: none)
+    int ctas;     // CTAs launched
+    bool pair;    // CTA-pair kernel (query groups of 128 columns)
     int64_t slots;
 };
+
+// Clusters of the pair kernel that can be resident at once on the current
+// device (0 if unknown, e.g. without a device): a persistent grid larger
+// than that would run its last clusters as a second wave.
+int pair_max_clusters() {
+    static int cache[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        cache[dev] = -1;
+        if (cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PairSmem::kBytes) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2);
+            cfg.blockDim = dim3(kPairThreads);
+            cfg.dynamicSmemBytes = PairSmem::kBytes;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, (void*)mla_decode_pair_kernel, &cfg) == cudaSuccess && n > 0)
+                cache[dev] = n;
+        }
+        cudaGetLastError();
+    }
+    return cache[dev] > 0 ? cache[dev] : 0;
+}
 
 int make_plan(const mla_decode_dims* d, Plan* pl) {
     int rc = validate_dims(d);
     if (rc != MLA_OK) return rc;
-    rc = resolve_ctas(d, &pl->G);
+    int sms = 0;
+    rc = resolve_ctas(d, &sms);
     if (rc != MLA_OK) return rc;
     pl->gr = make_grouping(d->num_heads, d->s_q);
-    pl->BG = d->batch * pl->gr.Hg;
-    pl->slots = max_slots(pl->G);
+    pl->pair = pl->gr.NG == kPairCols;
+    if (pl->pair) {
+        // one cluster of two CTAs per pair of SMs; the head groups of a
+        // request walk each range side by side on Hg clusters
+        int clusters = sms / 2 > 0 ? sms / 2 : 1;
+        const int resident = pair_max_clusters();
+        if (resident > 0 && clusters > resident) clusters = resident;
+        pl->G = clusters / pl->gr.Hg > 0 ? clusters / pl->gr.Hg : 1;
+        pl->BG = d->batch;
+        pl->plan_Hg = 1;
+        pl->shift = kStepShift;
+        pl->share = pl->gr.Hg;
+        pl->ctas = 2 * pl->G * pl->gr.Hg;
+        pl->slots = max_slots(pl->G) * pl->gr.Hg;
+    } else {
+        pl->G = sms;
+        pl->BG = d->batch * pl->gr.Hg;
+        pl->plan_Hg = pl->gr.Hg;
+        pl->shift = kPageShift;
+        pl->share = 1;
+        pl->ctas = sms;
+        pl->slots = max_slots(pl->G);
+    }
     return MLA_OK;
 }
 
@@ -115,6 +175,11 @@ int make_plan_gqa(const mla_gqa_dims* d, Plan* pl) {
     pl->gr.NG = kGqaHeadsPerGroup * d->s_q;
     pl->gr.Hg = d->num_kv_groups;
     pl->BG = d->batch * d->num_kv_groups;
+    pl->plan_Hg = pl->gr.Hg;
+    pl->shift = kPageShift;
+    pl->share = 1;
+    pl->ctas = pl->G;
+    pl->pair = false;
     pl->slots = max_slots(pl->G);
     return MLA_OK;
 }
@@ -189,13 +254,47 @@ int ensure_smem_attr() {
     return MLA_OK;
 }
 
+int launch_pair(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const CUtensorMap& qm,
+                cudaStream_t stream) {
+    {
+        static bool done[kMaxDevices] = {};
+        static std::mutex mu;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            if (cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     PairSmem::kBytes) != cudaSuccess)
+                return MLA_ERR_CUDA;
+            done[dev] = true;
+        }
+    }
+    // Clusters of two CTAs (compiled into the kernel), launched as a
+    // programmatic dependent of the schedule kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.ctas);
+    cfg.blockDim = dim3(kPairThreads);
+    cfg.dynamicSmemBytes = PairSmem::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, kvm, qm, p) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 template <int NG, class S>
 int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const CUtensorMap& qm,
                cudaStream_t stream) {
     int rc = ensure_smem_attr<NG, S>();
     if (rc != MLA_OK) return rc;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.G);
+    cfg.gridDim = dim3(pl.ctas);
     cfg.blockDim = dim3(FwdWarps<NG, S>::kThreads);
     cfg.dynamicSmemBytes = FwdSmem<NG, S>::kAlloc;
     cfg.stream = stream;
@@ -213,7 +312,7 @@ int launch_fwd(const Plan& pl, const FwdParams& p, const CUtensorMap& kvm, const
 
 // Query-column layout of the work items, for the kernels' item_col().
 struct ColMap {
-    int s_q, heads, run_rows, run_stride;
+    int s_q, heads, run_rows, run_stride, batch;
 };
 
 template <int kDvT>
@@ -233,12 +332,16 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
     c.NG = pl.gr.NG;
     c.Hg = pl.gr.Hg;
     c.G = pl.G;
-    c.BG = pl.BG;
+    c.BG = cm.batch * pl.gr.Hg;
     c.slots_cap = (int)pl.slots;
+    c.plan_BG = pl.BG;
+    c.plan_Hg = pl.plan_Hg;
+    c.shift = pl.shift;
+    c.share = pl.share;
     c.run_rows = cm.run_rows;
     c.run_stride = cm.run_stride;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.BG, pl.gr.NG);
+    cfg.gridDim = dim3(c.BG, pl.gr.NG);
     cfg.blockDim = dim3(kDvT / 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -254,7 +357,9 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-ColMap mla_colmap(const mla_decode_dims* d, const Plan& pl) { return ColMap{d->s_q, d->num_heads, pl.gr.NG, 0}; }
+ColMap mla_colmap(const mla_decode_dims* d, const Plan& pl) {
+    return ColMap{d->s_q, d->num_heads, pl.gr.NG, 0, d->batch};
+}
 
 // ---- scratch of the allocation-free entry point ----
 // One array per device, in this library's module; allocated by the driver when
@@ -414,8 +519,8 @@ int mla_decode_get_schedule(const mla_decode_dims* dims, const int32_t* cache_se
     const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
     const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
     mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
-        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.gr.Hg, pl.gr.NG, pl.G,
-        dims->max_blocks_per_seq, use_smem);
+        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.plan_Hg, pl.gr.NG, pl.G,
+        dims->max_blocks_per_seq, use_smem, pl.shift, pl.share);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -423,25 +528,28 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     int rc = validate_dims(dims);
     if (rc != MLA_OK) return rc;
     if (dims->num_sms <= 0 || seqlens == nullptr || schedule_host == nullptr) return MLA_ERR_INVALID_ARG;
-    const Grouping gr = make_grouping(dims->num_heads, dims->s_q);
-    const int G = dims->num_sms, BG = dims->batch * gr.Hg, mb = dims->max_blocks_per_seq;
+    Plan pl;
+    rc = make_plan(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    const Grouping gr = pl.gr;
+    const int G = pl.G, BG = pl.BG, Hg = pl.plan_Hg, sh = pl.shift, mb = dims->max_blocks_per_seq;
     int32_t* s = static_cast<int32_t*>(schedule_host);
     int32_t* prefix = s + prefix_offset_words(G, BG);
     int32_t* bginfo = s + bg_offset_words(G);
     int bad_len = 0;
     int64_t W = 0;
     for (int bg = 0; bg < BG; ++bg) {
-        const int L = seqlens[bg / gr.Hg];
+        const int L = seqlens[bg / Hg];
         if (!seqlen_in_range(L, mb)) bad_len = 1;
         prefix[bg] = (int32_t)W;
-        W += units_of(pages_of(clamp_seqlen(L, mb)));
+        W += units_of(blocks_of(clamp_seqlen(L, mb), sh));
     }
     prefix[BG] = (int32_t)W;
     const int64_t T = units_per_cta(W, G);
-    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, seqlens, gr.Hg, mb, s + kHdrWords + (size_t)k * kMetaWords);
+    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, seqlens, Hg, mb, sh, s + kHdrWords + (size_t)k * kMetaWords);
     int64_t slots = 0;
     for (int bg = 0; bg < BG; ++bg) {
-        const int ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, gr.Hg, mb), T);
+        const int ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, mb, sh), T);
         bginfo[kBgWords * bg] = (int32_t)slots;
         bginfo[kBgWords * bg + 1] = ns;
         if (ns > 1) slots += ns;
@@ -450,7 +558,7 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     s[kHdrMagic] = kSchedMagic;
     s[kHdrG] = G;
     s[kHdrBG] = BG;
-    s[kHdrHg] = gr.Hg;
+    s[kHdrHg] = Hg;
     s[kHdrNG] = gr.NG;
     s[kHdrSlots] = (int32_t)slots;
     s[kHdrT] = (int32_t)T;
@@ -458,6 +566,8 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     s[kHdrW] = (int32_t)W;
     s[kHdrBatch] = dims->batch;
     s[kHdrMaxBlocks] = mb;
+    s[kHdrShift] = sh;
+    s[kHdrShareHg] = pl.share;
     return MLA_OK;
 }
 
@@ -474,7 +584,8 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     CUtensorMap kvm, qm;
     rc = make_kv_map(&kvm, kv_cache, dims->num_blocks);
     if (rc != MLA_OK) return rc;
-    rc = make_q_map(&qm, q, dims->batch * pl.gr.N, pl.gr.NG);
+    // Q boxes: the group's rows (one CTA of a pair loads 64 of its 128)
+    rc = make_q_map(&qm, q, dims->batch * pl.gr.N, pl.pair ? kPairCols / 2 : pl.gr.NG);
     if (rc != MLA_OK) return rc;
     FwdParams p;
     p.sched = static_cast<const int32_t*>(schedule);
@@ -495,7 +606,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.causal = dims->causal;
     p.G = pl.G;
     p.BG = pl.BG;
-    p.Hg = pl.gr.Hg;
+    p.Hg = pl.pair ? pl.share : pl.gr.Hg;  // pair kernel: head groups walking each range
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
@@ -503,9 +614,10 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.run_rows = pl.gr.NG;
     p.run_stride = 0;
     p.kv_groups = 1;
-    rc = pl.gr.NG == 16   ? launch_fwd<16, ShapeMla>(pl, p, kvm, qm, st)
-         : pl.gr.NG == 32 ? launch_fwd<32, ShapeMla>(pl, p, kvm, qm, st)
-                          : launch_fwd<64, ShapeMla>(pl, p, kvm, qm, st);
+    rc = pl.pair            ? launch_pair(pl, p, kvm, qm, st)
+         : pl.gr.NG == 16   ? launch_fwd<16, ShapeMla>(pl, p, kvm, qm, st)
+         : pl.gr.NG == 32   ? launch_fwd<32, ShapeMla>(pl, p, kvm, qm, st)
+                            : launch_fwd<64, ShapeMla>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
     return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags, st);
@@ -543,8 +655,8 @@ int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_s
     const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
     const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
     mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
-        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.gr.Hg, pl.gr.NG, pl.G,
-        dims->max_blocks_per_seq, use_smem);
+        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.plan_Hg, pl.gr.NG, pl.G,
+        dims->max_blocks_per_seq, use_smem, pl.shift, pl.share);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -593,7 +705,7 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
     rc = pl.gr.NG == 16 ? launch_fwd<16, ShapeGqa>(pl, p, kvm, qm, st) : launch_fwd<32, ShapeGqa>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
-    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
+    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads, dims->batch},
                                          pl, schedule, workspace, out, lse, dims->flags, st);
 }
 
@@ -604,7 +716,7 @@ int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const
     if (rc != MLA_OK) return rc;
     if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
-    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads},
+    return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads, dims->batch},
                                          pl, schedule, workspace, out, lse, dims->flags,
                                          static_cast<cudaStream_t>(stream));
 }

@@ -1,7 +1,14 @@
 // Split-KV work partitioning for the persistent decode kernel.
 //
 // Work units: request b, head group g ("bg" = b * Hg + g) owns
-//   units(bg) = P_b + kItemOverhead   (P_b = ceil(L_b / 64) pages; 0 if P_b == 0)
+//   units(bg) = P_b + kItemOverhead   (P_b = ceil(L_b / 2^shift) token blocks of
+//                                       2^shift tokens; 0 if P_b == 0)
+// The one-CTA kernels walk 64-token pages (shift 6).  The CTA-pair kernel walks
+// steps of 128 tokens (shift 7, two pages per step), and builds its plan over
+// requests alone (Hg = 1 in the plan): each work range is then walked by the
+// request's head groups side by side, one cluster per group, so that the
+// groups read each page at about the same time and the repeats hit L2.
+// "Page" below means one such block.
 // The overhead stands for the per-item cost that does not scale with pages:
 // loading Q, filling the pipeline, the epilogue.  Units are laid out in bg
 // order and cut into G equal contiguous ranges of T units; CTA k owns
@@ -22,6 +29,8 @@
 namespace mla {
 
 constexpr int kPage = 64;
+constexpr int kPageShift = 6;      // one-CTA kernels: units of one 64-token page
+constexpr int kStepShift = 7;      // CTA-pair kernel: units of two pages
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kItemOverhead = 1;   // units charged per (request, head group)
@@ -45,6 +54,8 @@ enum HdrField {
     kHdrW = 8,
     kHdrBatch = 9,
     kHdrMaxBlocks = 10,
+    kHdrShift = 11,    // log2 of the tokens per unit (6 or 7)
+    kHdrShareHg = 12,  // head groups that walk every work range side by side (1: none)
 };
 constexpr int kMetaWords = 8;  // per CTA: begin_bg, begin_page, end_bg, end_page, first_split
 enum MetaField { kMetaBeginBg = 0, kMetaBeginPage = 1, kMetaEndBg = 2, kMetaEndPage = 3, kMetaFirstSplit = 4 };
@@ -59,12 +70,12 @@ __host__ __device__ inline int64_t schedule_words(int G, int BG) {
     return prefix_offset_words(G, BG) + BG + 1;
 }
 
-// Head grouping: N = heads * s_q query columns per request.  Up to 32 columns
-// go in one group (rounded up to 16 / 32 for the MMA N); more are cut into
-// groups of 32.
+// Head grouping: N = heads * s_q query columns per request.  Up to 64
+// columns go in one group of 16, 32 or 64 (the one-CTA kernel's MMA N); wider
+// requests are cut into groups of 128 columns for the CTA-pair kernel.
 struct Grouping {
     int N;   // heads * s_q
-    int NG;  // columns per group (MMA N): 16 or 32
+    int NG;  // columns per group: 16, 32, 64, or 128 (CTA pair)
     int Hg;  // groups per request
 };
 __host__ __device__ inline Grouping make_grouping(int heads, int s_q) {
@@ -76,9 +87,12 @@ __host__ __device__ inline Grouping make_grouping(int heads, int s_q) {
     } else if (gr.N <= 32) {
         gr.NG = 32;
         gr.Hg = 1;
-    } else {
+    } else if (gr.N <= 64) {
         gr.NG = 64;
-        gr.Hg = (gr.N + 63) / 64;
+        gr.Hg = 1;
+    } else {
+        gr.NG = 128;
+        gr.Hg = (gr.N + 127) / 128;
     }
     return gr;
 }
@@ -94,6 +108,8 @@ __host__ __device__ inline bool seqlen_in_range(int L, int max_blocks) {
     return L >= 0 && (int64_t)L <= (int64_t)max_blocks * kPage;
 }
 __host__ __device__ inline int pages_of(int L) { return (L + kPage - 1) / kPage; }
+// blocks of 2^shift tokens covering L tokens
+__host__ __device__ inline int blocks_of(int L, int shift) { return (L + (1 << shift) - 1) >> shift; }
 __host__ __device__ inline int64_t units_of(int P) { return P > 0 ? (int64_t)P + kItemOverhead : 0; }
 
 __host__ __device__ inline int64_t units_per_cta(int64_t W, int G) {
@@ -112,14 +128,15 @@ __host__ __device__ inline int find_bg(const int32_t* prefix, int BG, int64_t u)
     return lo;
 }
 
-// Pages of request-group bg under the clamp every kernel applies.
-__host__ __device__ inline int pages_of_bg(const int32_t* seqlens, int bg, int Hg, int max_blocks) {
-    return pages_of(clamp_seqlen(seqlens[bg / Hg], max_blocks));
+// Blocks of request-group bg under the clamp every kernel applies.
+__host__ __device__ inline int pages_of_bg(const int32_t* seqlens, int bg, int Hg, int max_blocks,
+                                           int shift = kPageShift) {
+    return blocks_of(clamp_seqlen(seqlens[bg / Hg], max_blocks), shift);
 }
 
 // (bg, page) position of unit u; u >= W maps to (BG, 0).
 __host__ __device__ inline void locate_unit(const int32_t* prefix, int BG, int64_t W, int64_t u,
-                                            const int32_t* seqlens, int Hg, int max_blocks,
+                                            const int32_t* seqlens, int Hg, int max_blocks, int shift,
                                             int* bg_out, int* page_out) {
     if (u >= W) {
         *bg_out = BG;
@@ -127,7 +144,7 @@ __host__ __device__ inline void locate_unit(const int32_t* prefix, int BG, int64
         return;
     }
     int bg = find_bg(prefix, BG, u);
-    int P = pages_of_bg(seqlens, bg, Hg, max_blocks);
+    int P = pages_of_bg(seqlens, bg, Hg, max_blocks, shift);
     int64_t p = u - (int64_t)prefix[bg] - kItemOverhead;
     if (p < 0) p = 0;
     if (p > P) p = P;
@@ -149,18 +166,18 @@ __host__ __device__ inline int num_splits_of(const int32_t* prefix, int bg, int 
 
 // Work range of CTA k: units [k*T, min((k+1)*T, W)).
 __host__ __device__ inline void cta_meta(const int32_t* prefix, int BG, int64_t W, int64_t T, int k,
-                                         const int32_t* seqlens, int Hg, int max_blocks,
+                                         const int32_t* seqlens, int Hg, int max_blocks, int shift,
                                          int32_t* meta) {
     int64_t u0 = (int64_t)k * T;
     int64_t u1 = u0 + T;
     if (u0 > W) u0 = W;
     if (u1 > W) u1 = W;
     int bb, bp, eb, ep;
-    locate_unit(prefix, BG, W, u0, seqlens, Hg, max_blocks, &bb, &bp);
-    locate_unit(prefix, BG, W, u1, seqlens, Hg, max_blocks, &eb, &ep);
+    locate_unit(prefix, BG, W, u0, seqlens, Hg, max_blocks, shift, &bb, &bp);
+    locate_unit(prefix, BG, W, u1, seqlens, Hg, max_blocks, shift, &eb, &ep);
     int first_split = 0;
     if (bb < BG) {
-        int P = pages_of_bg(seqlens, bb, Hg, max_blocks);
+        int P = pages_of_bg(seqlens, bb, Hg, max_blocks, shift);
         if (P > 0) {
             first_split = k - first_cta_of(prefix, bb, T);
             if (first_split < 0) first_split = 0;

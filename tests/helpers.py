@@ -82,10 +82,12 @@ def read_plan(buf: np.ndarray, G: int, BG: int):
     return hdr, meta, bginfo, prefix
 
 
-def walk_plan(meta, bginfo, seqlens, Hg, max_blocks):
-    """Items each CTA processes, exactly as the decode kernel walks its range:
-    list per CTA of (bg, p0, p1, unsplit, slot)."""
+def walk_plan(meta, bginfo, seqlens, Hg, max_blocks, shift=6):
+    """Items each work range holds, exactly as the decode kernels walk it:
+    list per range of (bg, p0, p1, unsplit, slot), in units of 2^shift tokens
+    (64-token pages, or the CTA-pair kernel's 128-token steps)."""
     BG = bginfo.shape[0]
+    unit = 1 << shift
     out = []
     for k in range(meta.shape[0]):
         bb, bp, eb, ep, fs = (int(x) for x in meta[k, :5])
@@ -95,7 +97,7 @@ def walk_plan(meta, bginfo, seqlens, Hg, max_blocks):
             cur = bg
             bg += 1
             L = min(max(int(seqlens[cur // Hg]), 0), max_blocks * 64)
-            P = (L + 63) // 64
+            P = (L + unit - 1) // unit
             p0 = bp if cur == bb else 0
             p1 = ep if cur == eb else P
             p1 = min(p1, P)

@@ -62,9 +62,13 @@ def test_sizes_need_valid_dims(lib):
     assert bd.mla_decode_workspace_bytes(d) == 2 * 148 * 16 * (512 + 1) * 4
     d32 = _dims(s_q=2)
     assert bd.mla_decode_workspace_bytes(d32) == 2 * 148 * 32 * 513 * 4
-    wide = _dims(s_q=2, num_heads=128, batch=32)  # 256 columns -> 4 groups of 64
-    assert bd.mla_decode_schedule_bytes(wide) == 4 * (16 + 8 * 148 + 3 * 32 * 4 + 1)
-    assert bd.mla_decode_workspace_bytes(wide) == 2 * 148 * 64 * 513 * 4
+    # 256 columns -> 2 groups of 128 on CTA pairs: 74 clusters, 37 ranges each
+    # walked by both groups; the plan has one row per request
+    wide = _dims(s_q=2, num_heads=128, batch=32)
+    assert bd.mla_decode_schedule_bytes(wide) == 4 * (16 + 8 * 37 + 3 * 32 + 1)
+    assert bd.mla_decode_workspace_bytes(wide) == (2 * 37 * 2) * 128 * 513 * 4
+    mid = _dims(s_q=2, num_heads=24)  # 48 columns -> one group of 64, one-CTA kernel
+    assert bd.mla_decode_workspace_bytes(mid) == 2 * 148 * 64 * 513 * 4
     for bad in (dict(batch=0), dict(s_q=0), dict(s_q=3), dict(num_heads=0), dict(num_blocks=0),
                 dict(max_blocks_per_seq=0), dict(num_sms=-1)):
         assert bd.mla_decode_schedule_bytes(_dims(**bad)) == 0, bad

@@ -24,10 +24,16 @@ def host_plan(seqlens, s_q, heads, G, max_blocks=None):
     n = bd.mla_decode_schedule_bytes(d)
     buf = torch.zeros(n, dtype=torch.uint8)
     bd.mla_decode_get_schedule_host(d, seqlens, buf)
-    Hg = 1 if heads * s_q <= 64 else (heads * s_q + 63) // 64
-    BG = B * Hg
-    hdr, meta, bginfo, prefix = helpers.read_plan(buf.numpy(), G, BG)
-    return dict(hdr=hdr, meta=meta, bginfo=bginfo, prefix=prefix, Hg=Hg, BG=BG, G=G,
+    N = heads * s_q
+    words = buf.numpy().view(np.int32)
+    if N <= 64:  # one-CTA kernels: one plan row per request-group, 64-token pages
+        Hg, BG, Gp, shift, share = 1, B, G, 6, 1
+    else:        # CTA pairs: one row per request, 128-token steps, ranges shared by the groups
+        share = (N + 127) // 128
+        Hg, BG, Gp, shift = 1, B, max(1, max(1, G // 2) // share), 7
+    assert (int(words[1]), int(words[2]), int(words[3]), int(words[11]), int(words[12])) == (Gp, BG, Hg, shift, share)
+    hdr, meta, bginfo, prefix = helpers.read_plan(buf.numpy(), Gp, BG)
+    return dict(hdr=hdr, meta=meta, bginfo=bginfo, prefix=prefix, Hg=Hg, BG=BG, G=Gp, shift=shift, share=share,
                 seqlens=seqlens.numpy(), max_blocks=max_blocks)
 
 
@@ -36,8 +42,9 @@ def check_invariants(pl):
     hdr, meta, bginfo = pl["hdr"], pl["meta"], pl["bginfo"]
     assert hdr[0] == 0x4D4C4144 and hdr[1] == G and hdr[2] == BG and hdr[3] == Hg
     T = int(hdr[6])
-    items = helpers.walk_plan(meta, bginfo, seq, Hg, mb)
-    pages = [(min(max(int(seq[bg // Hg]), 0), mb * 64) + 63) // 64 for bg in range(BG)]
+    unit = 1 << pl["shift"]
+    items = helpers.walk_plan(meta, bginfo, seq, Hg, mb, pl["shift"])
+    pages = [(min(max(int(seq[bg // Hg]), 0), mb * 64) + unit - 1) // unit for bg in range(BG)]
     covered = [np.zeros(P, dtype=np.int64) for P in pages]
     pieces = [[] for _ in range(BG)]
     for k, its in enumerate(items):
@@ -79,11 +86,11 @@ def test_plan_of_each_workload(name):
     items = check_invariants(pl)
     busy = sum(1 for its in items if its)
     W = int(pl["hdr"][8])
-    assert busy == min(148, -(-W // int(pl["hdr"][6])))
+    assert busy == min(pl["G"], -(-W // int(pl["hdr"][6])))
 
 
 @pytest.mark.parametrize("G", [1, 2, 7, 148, 300])
-@pytest.mark.parametrize("heads,s_q", [(16, 1), (16, 2), (1, 1), (3, 2), (24, 2), (128, 2)])
+@pytest.mark.parametrize("heads,s_q", [(16, 1), (16, 2), (1, 1), (3, 2), (24, 2), (40, 2), (128, 1), (128, 2)])
 def test_plan_random_ragged(G, heads, s_q):
     rng = np.random.default_rng(G * 1000 + heads * 10 + s_q)
     lens = rng.integers(0, 3000, size=int(rng.integers(1, 40))).tolist()
