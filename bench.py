@@ -2,9 +2,12 @@
 """MLA decode benchmark: us/call and KV GB/s of one decode step on B200.
 
 A step is one pass of the whole hot path over one batch: the split-KV
-schedule, the persistent decode kernel and the LSE combine, all launched
-through the C ABI (libmla_decode.so) and captured once as a CUDA graph
-that every timed step replays.  Default workload: batch 16, s_q 1,
+schedule, the persistent decode kernel and the LSE combine, launched by one
+mla_decode_fwd call through the C ABI (libmla_decode.so) with
+MLA_FLAG_INLINE_PLAN (the decode kernel builds the schedule from the lengths
+in its prologue; for the 128-column CTA-pair kernel the call enqueues the
+schedule kernel first), captured once as a CUDA graph that every timed step
+replays.  Default workload: batch 16, s_q 1,
 16 heads, KV length 65536 (1.21 GB of latent cache per step, larger than L2,
 so no flush is needed between steps).
 
@@ -66,6 +69,15 @@ def parse_args():
 
 
 # ---------------------------------------------------------------- accounting
+def flush_l2(flush: torch.Tensor, i: int) -> None:
+    """Untimed, before a timed replay: overwrite L2 with a buffer larger than
+    it, then hold the GPU for ~50 us so that the host has enqueued the start
+    event and the replay before the GPU reaches them; the timed interval then
+    holds the replay's own execution and no host enqueue latency."""
+    flush.fill_(i & 0xFF)
+    torch.cuda._sleep(100_000)
+
+
 def kv_tokens(seqlens: torch.Tensor) -> int:
     return int(seqlens.clamp(min=0).to(torch.int64).sum())
 
@@ -334,7 +346,8 @@ def workload_config(w, d, n_gpus):
         "page_size": 64, "causal": w.causal, "softmax_scale": "192^-0.5",
         "kv_bytes_per_step": byt["kv"],
         "l2": "inputs larger than L2 (%.2f GB KV per step): no flush" % (byt["kv"] / 1e9)
-              if byt["kv"] > 2 * 126e6 else "L2 flushed between steps (256 MB write, untimed)",
+              if byt["kv"] > 2 * 126e6 else "L2 flushed between steps (256 MB write and a 50 us GPU wait, untimed)",
+        "plan": "built every step from cache_seqlens (MLA_FLAG_INLINE_PLAN)",
         "parallelism": "dp%d: independent request batches per GPU, no collective" % n_gpus,
     }
 
@@ -360,7 +373,10 @@ def run_ours(args, w):
     sl = d["cache_seqlens"].to(dev)
     B, s_q, h = w.batch, w.s_q, w.heads
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    dims = bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms)
+    # The step is one mla_decode_fwd call that builds its split-KV plan from
+    # the lengths itself (MLA_FLAG_INLINE_PLAN); mla_decode_get_schedule runs
+    # once, before the warm-up, to clear the new buffer's status word.
+    dims = bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms, bd.MLA_FLAG_INLINE_PLAN)
     sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
     ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
     out = torch.empty(B, s_q, h, 512, dtype=torch.bfloat16, device=dev)
@@ -375,10 +391,11 @@ def run_ours(args, w):
     # The decode kernel and the combine are launched as programmatic
     # dependents (PDL) of the kernel before them, so the timed loop records
     # no events between the kernels of a step.
-    dims_nc = bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms, bd.MLA_FLAG_NO_COMBINE)
+    dims_nc = bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms,
+                           bd.MLA_FLAG_NO_COMBINE | bd.MLA_FLAG_INLINE_PLAN)
+    bd.mla_decode_get_schedule(dims, sl, sched, stream)
 
     def step():
-        bd.mla_decode_get_schedule(dims, sl, sched, stream)
         bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, stream)
 
     def decode_only():
@@ -400,7 +417,6 @@ def run_ours(args, w):
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
         with torch.cuda.graph(g_step, stream=cap):
-            bd.mla_decode_get_schedule(dims, sl, sched, cap)
             bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, cap)
         with torch.cuda.graph(g_dec, stream=cap):
             bd.mla_decode_fwd(dims_nc, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, cap)
@@ -423,7 +439,7 @@ def run_ours(args, w):
     t_start.record(stream)
     for i in range(args.steps):
         if flush is not None:
-            flush.fill_(i & 0xFF)
+            flush_l2(flush, i)
             steps_ev[i][0].record(stream)
         g_step.replay()
         if flush is not None:
@@ -445,7 +461,7 @@ def run_ours(args, w):
             for _ in range(args.steps)]
     for i in range(args.steps):
         if flush is not None:
-            flush.fill_(i & 0xFF)
+            flush_l2(flush, i)
         kern[i][0].record(stream)
         g_dec.replay()
         kern[i][1].record(stream)
@@ -555,7 +571,6 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
 
     def step(st):
         in_d.copy_(in_h, non_blocking=True)
-        bd.mla_decode_get_schedule(dims, sl, sched, st)
         bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
         res_h.copy_(res_d, non_blocking=True)
 
@@ -599,7 +614,7 @@ def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
 
 
 def measure_case(w, d, dev, steps, warmup, hbm_peak, tf_peak):
-    """One named workload on this GPU: the step (schedule + decode + combine)
+    """One named workload on this GPU: the step (plan + decode + combine)
     and the decode kernel alone, each graph-replayed with CUDA events around
     every replay (L2 flushed before each replay, untimed, where the KV fits
     twice into L2); median and best per call.  Then one more step in bf16 and
@@ -614,7 +629,8 @@ def measure_case(w, d, dev, steps, warmup, hbm_peak, tf_peak):
     sl = d["cache_seqlens"].to(dev)
     B, s_q, h = w.batch, w.s_q, w.heads
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    mk = lambda flags=0: bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms, flags)
+    mk = lambda flags=0: bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, num_sms,
+                                      flags | bd.MLA_FLAG_INLINE_PLAN)
     dims, dims_nc, dims_f32 = mk(), mk(bd.MLA_FLAG_NO_COMBINE), mk(bd.MLA_FLAG_FP32_OUT)
     sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
     ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
@@ -632,22 +648,21 @@ def measure_case(w, d, dev, steps, warmup, hbm_peak, tf_peak):
         cap = torch.cuda.Stream(dev)
         cap.wait_stream(stream)
         with torch.cuda.stream(cap):
-            bd.mla_decode_get_schedule(dims, sl, sched, cap)
+            bd.mla_decode_get_schedule(dims, sl, sched, cap)  # clears the status word once
             bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, scale, out, lse, cap)
             with torch.cuda.graph(g, stream=cap):
-                if dm is dims:
-                    bd.mla_decode_get_schedule(dims, sl, sched, cap)
                 bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, scale, out, lse, cap)
         stream.wait_stream(cap)
         graphs.append(g)
     times = []
     for g in graphs:
+        n_it = max(3, warmup) + steps
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_it)]
         ev = []
-        for i in range(max(3, warmup) + steps):
+        for i in range(n_it):
+            a, b = evs[i]
             if flush is not None:
-                flush.fill_(i & 0xFF)
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
+                flush_l2(flush, i)
             a.record(stream)
             g.replay()
             b.record(stream)
@@ -661,7 +676,6 @@ def measure_case(w, d, dev, steps, warmup, hbm_peak, tf_peak):
     med = lambda t: statistics.median(t)
 
     # parity, every row: the bf16 output and the fp32 output before the cast
-    bd.mla_decode_get_schedule(dims, sl, sched, stream)
     bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, scale, out, lse, stream)
     torch.cuda.synchronize()
     o16 = out.float().cpu().numpy().reshape(-1, 512)
@@ -734,8 +748,9 @@ def run_sweep(args):
             d = workloads.build(B, 1, 16, ("fixed", L), seed=3000 + B, pool_device="cuda")
             q, kv = d["q"].to(dev), d["kv_cache"]
             bt, sl = d["block_table"].to(dev), d["cache_seqlens"].to(dev)
-            dims = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0)
-            dnc = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0, bd.MLA_FLAG_NO_COMBINE)
+            dims = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0, bd.MLA_FLAG_INLINE_PLAN)
+            dnc = bd.make_dims(B, 1, 16, kv.shape[0], bt.shape[1], False, 0,
+                               bd.MLA_FLAG_NO_COMBINE | bd.MLA_FLAG_INLINE_PLAN)
             sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
             ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
             out = torch.empty(B, 1, 16, 512, dtype=torch.bfloat16, device=dev)
@@ -743,8 +758,9 @@ def run_sweep(args):
             byt = algorithmic_bytes(d["cache_seqlens"], 1, 16)
             use_flush = byt["total"] < (512 << 20)
 
+            bd.mla_decode_get_schedule(dims, sl, sched, stream)  # clears the status word once
+
             def step(st, dm=dims):
-                bd.mla_decode_get_schedule(dm, sl, sched, st)
                 bd.mla_decode_fwd(dm, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
 
             times = []
@@ -758,11 +774,12 @@ def run_sweep(args):
                         step(cap, dm)
                 stream.wait_stream(cap)
                 ts = []
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(3 + args.steps)]
                 for i in range(3 + args.steps):
+                    a, b = evs[i]
                     if use_flush:
-                        flush.fill_(i & 255)
-                    a = torch.cuda.Event(enable_timing=True)
-                    b = torch.cuda.Event(enable_timing=True)
+                        flush_l2(flush, i)
                     a.record(stream)
                     g.replay()
                     b.record(stream)
@@ -798,8 +815,9 @@ def run_gqa_bench(args):
     d = workloads.build_gqa(B, s_q, groups, ("fixed", L), seed=1005, causal=True, pool_device="cuda")
     q, kv = d["q"].to(dev), d["kv_cache"]
     bt, sl = d["block_table"].to(dev), d["cache_seqlens"].to(dev)
-    dims = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0)
-    dnc = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0, bd.MLA_FLAG_NO_COMBINE)
+    dims = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0, bd.MLA_FLAG_INLINE_PLAN)
+    dnc = bd.make_gqa_dims(B, s_q, groups, kv.shape[0], bt.shape[1], True, 0,
+                           bd.MLA_FLAG_NO_COMBINE | bd.MLA_FLAG_INLINE_PLAN)
     sched = torch.empty(bd.mla_gqa_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
     ws = torch.empty(bd.mla_gqa_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
     out = torch.empty(B, s_q, h, 128, dtype=torch.bfloat16, device=dev)
@@ -809,8 +827,9 @@ def run_gqa_bench(args):
     total_bytes = kv_bytes + q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
     flops = 2 * h * s_q * tokens * (192 + 128)
 
+    bd.mla_gqa_decode_get_schedule(dims, sl, sched, stream)  # clears the status word once
+
     def step(st, dm):
-        bd.mla_gqa_decode_get_schedule(dm, sl, sched, st)
         bd.mla_gqa_decode_fwd(dm, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
 
     times = []

@@ -85,6 +85,19 @@ extern "C" {
  * accumulation itself.  Applies to mla_decode_fwd, mla_decode_combine and
  * the GQA-path calls; pass the same flags to both when combining separately. */
 #define MLA_FLAG_FP32_OUT 0x4
+/* mla_decode_fwd (and mla_gqa_decode_fwd) build the split-KV plan themselves
+ * from cache_seqlens, so a step needs no mla_decode_get_schedule call: for
+ * query groups of up to 64 columns (heads * s_q <= 64; every GQA shape) the
+ * decode kernel computes its own work range in its prologue, which removes
+ * the schedule kernel's launch from the step, and writes the same plan
+ * mla_decode_get_schedule would into `schedule`; for wider groups, or more
+ * request-groups than its shared memory holds (batch * groups > 18,384 for
+ * MLA, > 10,192 for GQA), the call enqueues the schedule kernel before the
+ * decode kernel.  The status word is not cleared by these calls: call
+ * mla_decode_get_schedule once on a new buffer to clear it, after which it
+ * collects the faults of every later call until the next
+ * mla_decode_get_schedule.  Pass the same flags to mla_decode_combine. */
+#define MLA_FLAG_INLINE_PLAN 0x8
 
 typedef struct mla_decode_dims {
     int32_t batch;              /* B >= 1 */
@@ -136,11 +149,13 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* cac
  *   out          bf16 [batch][s_q][num_heads][512] (fp32 with MLA_FLAG_FP32_OUT)
  *   lse          fp32 [batch][num_heads][s_q]  (natural log; -inf if nothing is visible)
  *   schedule     from mla_decode_get_schedule with the same dims and lengths
+ *                (with MLA_FLAG_INLINE_PLAN: any buffer of
+ *                mla_decode_schedule_bytes(dims) bytes; the call writes the plan)
  *   workspace    mla_decode_workspace_bytes(dims) bytes, no initialisation needed
  * Enqueues the persistent decode kernel and then (unless MLA_FLAG_NO_COMBINE)
  * the combine kernel on `stream`.  A request whose visible range is empty
  * gets out = 0 and lse = -inf. */
-int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* workspace,
+int mla_decode_fwd(const mla_decode_dims* dims, void* schedule, void* workspace,
                    const void* q, const void* kv_cache, const int32_t* block_table,
                    const int32_t* cache_seqlens, float softmax_scale, void* out, float* lse,
                    void* stream);
@@ -153,7 +168,8 @@ int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const 
                        void* out, float* lse, void* stream);
 
 /* Copies the device status word (OR of MLA_STATUS_* bits since the last
- * mla_decode_get_schedule) to *host_status.  Synchronous: waits for the copy
+ * mla_decode_get_schedule, including those of every MLA_FLAG_INLINE_PLAN call
+ * since) to *host_status.  Synchronous: waits for the copy
  * on the legacy default stream, so call it after the work it should cover has
  * finished (e.g. after synchronising the stream that ran it). */
 int mla_decode_get_status(const void* schedule, int32_t* host_status);
@@ -232,7 +248,7 @@ size_t mla_gqa_decode_schedule_bytes(const mla_gqa_dims* dims);
 size_t mla_gqa_decode_workspace_bytes(const mla_gqa_dims* dims);
 int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_seqlens, void* schedule,
                                 void* stream);
-int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* workspace, const void* q,
+int mla_gqa_decode_fwd(const mla_gqa_dims* dims, void* schedule, void* workspace, const void* q,
                        const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
                        float softmax_scale, void* out, float* lse, void* stream);
 int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,

@@ -32,6 +32,7 @@ MLA_STATUS_SMEM_ALIGN = 0x10
 MLA_FLAG_NO_COMBINE = 0x1
 MLA_FLAG_TEST_STALL = 0x2
 MLA_FLAG_FP32_OUT = 0x4
+MLA_FLAG_INLINE_PLAN = 0x8
 
 PAGE_SIZE = 64
 D_QK = 576
@@ -244,17 +245,19 @@ class MlaDecoder:
     ``plan(cache_seqlens)`` builds the split-KV schedule (once per decode step);
     ``__call__`` runs the decode kernel + combine and returns (out, lse).
     With ``fp32_out`` the output is fp32 (MLA_FLAG_FP32_OUT): the result before
-    any rounding to bf16.
+    any rounding to bf16.  With ``inline_plan`` (MLA_FLAG_INLINE_PLAN) every
+    call builds the plan itself; ``plan()`` is then needed once, to clear the
+    status word of the new buffer.
     """
 
     def __init__(self, batch: int, s_q: int, num_heads: int, num_blocks: int,
                  max_blocks_per_seq: int, causal: bool = False, num_sms: int = 0,
-                 device: Optional[torch.device] = None, fp32_out: bool = False):
+                 device: Optional[torch.device] = None, fp32_out: bool = False, inline_plan: bool = False):
         self.device = torch.device(device or "cuda")
         if num_sms == 0:
             num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.dims = make_dims(batch, s_q, num_heads, num_blocks, max_blocks_per_seq, causal, num_sms,
-                              MLA_FLAG_FP32_OUT if fp32_out else 0)
+                              (MLA_FLAG_FP32_OUT if fp32_out else 0) | (MLA_FLAG_INLINE_PLAN if inline_plan else 0))
         sb = mla_decode_schedule_bytes(self.dims)
         wb = mla_decode_workspace_bytes(self.dims)
         if sb == 0 or wb == 0:
@@ -350,12 +353,12 @@ class GqaDecoder:
 
     def __init__(self, batch: int, s_q: int, num_kv_groups: int, num_blocks: int, max_blocks_per_seq: int,
                  causal: bool = False, num_sms: int = 0, device: Optional[torch.device] = None,
-                 fp32_out: bool = False):
+                 fp32_out: bool = False, inline_plan: bool = False):
         self.device = torch.device(device or "cuda")
         if num_sms == 0:
             num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.dims = make_gqa_dims(batch, s_q, num_kv_groups, num_blocks, max_blocks_per_seq, causal, num_sms,
-                                  MLA_FLAG_FP32_OUT if fp32_out else 0)
+                                  (MLA_FLAG_FP32_OUT if fp32_out else 0) | (MLA_FLAG_INLINE_PLAN if inline_plan else 0))
         sb = mla_gqa_decode_schedule_bytes(self.dims)
         wb = mla_gqa_decode_workspace_bytes(self.dims)
         if sb == 0 or wb == 0:

@@ -161,6 +161,9 @@ constexpr float kLn2 = 0.693147180559945309f;
 // 228.9 us, 1 page ahead 212.5, 2 pages 214.6, 4 pages 218.5, 8 pages 271.7.
 // Short work items gain nothing and lose a little, so only items of at least
 // kPrefetchMinPages pages prefetch.
+// Measured as well: prefetching every page of an item into L2 when the item
+// starts, on steps whose pages fit L2 (bs16 x 4K: 30.8 -> 35-37 us; 1 x 1K:
+// 16.5 -> 18.4 us): the bulk prefetches delay the page loads behind them.
 constexpr int kPrefetchPages = 1;
 constexpr int kPrefetchMinPages = 16;
 
@@ -202,7 +205,7 @@ struct Tracer {
     __device__ void ev(unsigned tag) {
         if (on && cta < kTraceCtas && n < kTraceCap)
             g_mla_trace[cta][role][n] = (static_cast<unsigned long long>(tag) << 56) |
-                                        (global_timer_ns() & 0x00FFFFFFFFFFFFFFull);
+                                        (stamp_timer_ns() & 0x00FFFFFFFFFFFFFFull);
         ++n;
     }
     __device__ ~Tracer() {
@@ -211,13 +214,37 @@ struct Tracer {
 };
 #define MLA_TRACE_DECL(role) Tracer tracer_(role)
 #define MLA_TRACE_EV(tag) tracer_.ev(tag)
+// Kernel-level stamps: per decode CTA [entry, plan readable, setup done, -,
+// TMEM released, GEMM1 / GEMM2 / softmax role returned];
+// for the whole step [schedule entry, schedule exit, first combine entry,
+// first combine past its wait, last combine exit] (min / max over blocks).
+__device__ unsigned long long g_mla_trace_k[kTraceCtas][8];
+__device__ unsigned long long g_mla_trace_step[8];
+__device__ unsigned long long g_mla_trace_comb[64][64];  // combine CTA (bg, column) exit
+#define MLA_TRACE_K(slot) MLA_TRACE_K_BY(slot, 0)
+#define MLA_TRACE_K_BY(slot, thread)                                           \
+    do {                                                                       \
+        if (threadIdx.x == (thread) && blockIdx.x < kTraceCtas)                \
+            g_mla_trace_k[blockIdx.x][slot] = stamp_timer_ns();                \
+    } while (0)
+#define MLA_TRACE_STEP_MIN(slot) \
+    do { if (threadIdx.x == 0) atomicMin(&g_mla_trace_step[slot], stamp_timer_ns()); } while (0)
+#define MLA_TRACE_STEP_MAX(slot) \
+    do { if (threadIdx.x == 0) atomicMax(&g_mla_trace_step[slot], stamp_timer_ns()); } while (0)
 #else
 #define MLA_TRACE_DECL(role)
 #define MLA_TRACE_EV(tag)
+#define MLA_TRACE_K(slot)
+#define MLA_TRACE_K_BY(slot, thread)
+#define MLA_TRACE_STEP_MIN(slot)
+#define MLA_TRACE_STEP_MAX(slot)
 #endif
 
 struct FwdParams {
     const int32_t* sched;
+    // Non-null: the kernel builds the plan itself from the lengths and writes
+    // it here (the schedule buffer); null: it reads the plan in `sched`.
+    int32_t* plan_out;
     const int32_t* block_table;
     const int32_t* seqlens;
     const uint8_t* kv;  // page pool base (for L2 prefetch)
@@ -264,6 +291,7 @@ struct CombineParams {
     // plan has one row per request-group; else one row per request, and split
     // i of group g sits in slot (base + i) * share + g).
     int plan_BG, plan_Hg, shift, share;
+    int plan_in_decode;  // the decode kernel built the plan (read it only after the wait)
 };
 
 // ------------------------------------------------------------------ layout
@@ -302,7 +330,10 @@ struct FwdSmem {
     static constexpr int kBarOff = kVoteOff + 2 * 8 * 4;
     static constexpr int kNumBars = 32;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
-    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kPlanMetaOff = kMiscOff + 16;         // this CTA's plan row (+2 words), when built in the kernel
+    static constexpr int kBytes = kPlanMetaOff + (kMetaWords + 8) * 4;
+    // largest plan (request-groups) the kernel builds itself: prefix + scan state in one stage
+    static constexpr int kInlinePlanMaxBG = kStageBytes / 4 - 48;  // prefix (BG + 1) + 32 warp totals
     // Slack to align the base to 1 KB where it fits; without it the kernel
     // checks that the dynamic shared memory base is 1 KB aligned.
     static constexpr int kAlignSlack = kBytes + 1024 <= 227 * 1024 ? 1024 : 0;
@@ -375,18 +406,19 @@ struct Item {
 };
 
 struct WorkIter {
-    int bg, begin_bg, begin_page, end_bg, end_page, first_split;
+    int bg, begin_bg, begin_page, end_bg, end_page;
 
+    // meta: this CTA's row of the plan, in the schedule buffer or (plan built
+    // by the kernel itself) in shared memory.
     __device__ void init(const int32_t* meta) {
-        begin_bg = __ldg(meta + kMetaBeginBg);
-        begin_page = __ldg(meta + kMetaBeginPage);
-        end_bg = __ldg(meta + kMetaEndBg);
-        end_page = __ldg(meta + kMetaEndPage);
-        first_split = __ldg(meta + kMetaFirstSplit);
+        begin_bg = meta[kMetaBeginBg];
+        begin_page = meta[kMetaBeginPage];
+        end_bg = meta[kMetaEndBg];
+        end_page = meta[kMetaEndPage];
         bg = begin_bg;
     }
 
-    __device__ bool next(const FwdParams& p, const int32_t* bginfo, Item& it) {
+    __device__ bool next(const FwdParams& p, Item& it) {
         while (bg <= end_bg && bg < p.BG) {
             const int cur = bg++;
             const int b = cur / p.Hg;
@@ -406,8 +438,9 @@ struct WorkIter {
             it.unsplit = (p0 == 0 && p1 == P);
             it.slot = -1;
             if (!it.unsplit) {
-                const int s = __ldg(bginfo + kBgWords * cur) + ((cur == begin_bg) ? first_split : 0);
-                it.slot = (s >= 0 && s < p.slots_cap) ? s : -1;
+                // first item: slot 2k; last item: slot 2k + 1 (see cta_slot)
+                const int s = cta_slot(blockIdx.x, cur == begin_bg);
+                it.slot = s < p.slots_cap ? s : -1;
             }
             return true;
         }
@@ -519,7 +552,7 @@ __device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const float (&v)
 // ------------------------------------------------------------------ roles
 template <int NG, class S>
 __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map,
-                             const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+                             const FwdParams& p, const int32_t* meta,
                              uint8_t* smem, const Ctl& ctl) {
     using L = FwdSmem<NG, S>;
     const uint32_t kv_s = smem_addr(smem + L::kKvOff);
@@ -534,7 +567,7 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     bool stall = p.test_stall != 0;
     bool ok = true;
     MLA_TRACE_DECL(0);
-    while (ok && it.next(p, bginfo, item)) {
+    while (ok && it.next(p, item)) {
         MLA_TRACE_EV(kTrItem);
         ok = wait_bounded(bar0 + 8 * kQEmpty, (q_it & 1) ^ 1, ctl);
         if (!ok) break;
@@ -605,7 +638,7 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
 // advances 32 B inside the 128-byte swizzle atom.  k-step i accumulates into
 // the accumulator of its issuer.
 template <int NG, class S>
-__device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+__device__ void run_gemm1(const FwdParams& p, const int32_t* meta,
                           uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
     using L = FwdSmem<NG, S>;
     constexpr uint32_t kIdescS = idesc_bf16_f32(64, NG, 0, 0);
@@ -624,7 +657,7 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
     // units): build them once and add offsets.
     const uint64_t a_desc0 = smem_desc(kv_s, 16, 1024, kSwizzle128);
     const uint64_t b_desc0 = smem_desc(q_s, 16, 1024, kSwizzle128);
-    while (ok && it.next(p, bginfo, item)) {
+    while (ok && it.next(p, item)) {
         ok = wait_bounded(bar0 + 8 * kQFull, q_it & 1, ctl);
         if (!ok) break;
         for (int j = item.p0; j < item.p1; ++j) {
@@ -670,7 +703,7 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta, const int32_t
 // 8 KB on, 8-token groups 1 KB apart); P^T is MN-major with NG columns per
 // token row.  k-outer order keeps consecutive MMAs on different accumulators.
 template <int NG, class S>
-__device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+__device__ void run_gemm2(const FwdParams& p, const int32_t* meta,
                           uint8_t* smem, uint32_t tmem, const Ctl& ctl, int issuer) {
     constexpr int kIssuers = FwdWarps<NG, S>::kG2Issuers;
     constexpr int kChunksPer = S::kVChunks / kIssuers;  // d_v chunks of 128 per issuer
@@ -691,7 +724,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
 #endif
     const uint64_t a_desc0 = smem_desc(kv_s, L::kBoxBytes, 1024, kSwizzle128);
     const uint64_t b_desc0 = smem_desc(p_s, L::kPBytes, 8 * NP * 2, kPSwizzle);
-    while (ok && it.next(p, bginfo, item)) {
+    while (ok && it.next(p, item)) {
         for (int j = item.p0; j < item.p1; ++j) {
             const int st = s_it % L::kStages;  // KV stage of the page (holds its P^T)
             const int pb = s_it & 1;            // P^T handoff barriers
@@ -730,7 +763,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta, const int32_t
 }
 
 template <int NG, class S>
-__device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32_t* bginfo,
+__device__ void run_softmax(const FwdParams& p, const int32_t* meta,
                             uint8_t* smem, uint32_t tmem, const Ctl& ctl) {
     using L = FwdSmem<NG, S>;
     using Wp = FwdWarps<NG, S>;
@@ -783,7 +816,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
     Item item;
     uint32_t s_it = 0, item_it = 0, out_it = 0, max_it = 0;
     bool ok = true;
-    while (ok && it.next(p, bginfo, item)) {
+    while (ok && it.next(p, item)) {
         int lvis[W];                                      // visible length of each own column
 #pragma unroll
         for (int i = 0; i < W; ++i) {
@@ -1193,6 +1226,137 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta, const int32
         if (gt == 0) bulk_wait_all();  // output copies complete before the CTA exits
 }
 
+// Block-wide inclusive scan of one int per thread (blockDim.x a multiple of
+// 32, at most 1024); warp_tot holds 32 ints of shared memory.
+__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int r = v + (warp > 0 ? warp_tot[warp - 1] : 0);
+    __syncthreads();
+    return r;
+}
+
+// The split-KV plan built inside the decode kernel from the lengths alone:
+// the same plan mla_decode_schedule_kernel writes (schedule.cuh), without its
+// launch.  The unit prefix over request-groups goes to `scratch` (BG + 1 words
+// plus 32 of warp totals, in a page stage that no copy has targeted yet);
+// this CTA's range to plan_s[0..7], with plan_s[8], plan_s[9] as the split
+// count and bad-length flag for the header.  Each CTA also writes its share of
+// the plan to the schedule buffer, for the combine kernel and for inspection:
+// its meta row; the rows of the request-groups whose first page it holds (CTA
+// 0 takes those with no pages); and CTA 0 the header and the prefix.  The
+// header's status word is left alone, so faults accumulate until the next
+// mla_decode_get_schedule clears it.  Every thread takes part; three block
+// barriers when BG fits one pass of the CTA's threads, the last one at the
+// end, after which the scratch stage is free.
+__device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, int32_t* plan_s) {
+    const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int k = blockIdx.x, G = gridDim.x, BG = p.BG, Hg = p.Hg, mb = p.max_blocks;
+    int32_t* prefix = scratch;
+    int32_t* warp_tot = scratch + BG + 1;
+    int32_t* meta_s = plan_s;
+    int32_t* total_slots = plan_s + kMetaWords;
+    int32_t* bad = plan_s + kMetaWords + 1;
+    if (tid == 0) {
+        *total_slots = 0;
+        *bad = 0;
+    }
+    // Unit prefix, one pass of nthr request-groups at a time: a warp scan by
+    // shuffles, then every thread adds the totals of the warps before it.
+    int carry = 0;
+    bool any_bad = false;
+    for (int base = 0; base < BG; base += nthr) {
+        const int bg = base + tid;
+        int v = 0;
+        if (bg < BG) {
+            const int L = __ldg(p.seqlens + bg / Hg);
+            any_bad |= !seqlen_in_range(L, mb);
+            v = (int)units_of(blocks_of(clamp_seqlen(L, mb), kPageShift));
+        }
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[warp] = x;
+        __syncthreads();
+        int before = carry, total = carry;
+        for (int w = 0; w < nwarps; ++w) {
+            const int t = warp_tot[w];
+            before += w < warp ? t : 0;
+            total += t;
+        }
+        if (bg < BG) prefix[bg] = before + x - v;
+        carry = total;
+        if (base + nthr < BG) __syncthreads();  // warp_tot is reused by the next pass
+    }
+    const int64_t W = carry;
+    if (tid == 0) prefix[BG] = (int)W;
+    if (any_bad) *bad = 1;
+    __syncthreads();
+    const int64_t T = units_per_cta(W, G);
+    if (tid == 0) {
+        cta_meta(prefix, BG, W, T, k, meta_s);
+        int32_t* row = p.plan_out + kHdrWords + (size_t)k * kMetaWords;
+        for (int i = 0; i < kMetaWords; ++i) row[i] = meta_s[i];
+    }
+    int32_t* bginfo = p.plan_out + bg_offset_words(G);
+    int my_slots = 0;
+    for (int bg = tid; bg < BG; bg += nthr) {
+        const int P = pages_in_prefix(prefix, bg);
+        const int ns = num_splits_of(prefix, bg, P, T);
+        if (ns > 1) my_slots += ns;
+        int owner = P > 0 ? first_cta_of(prefix, bg, T) : 0;
+        if (owner > G - 1) owner = G - 1;
+        if (owner == k) {
+            bginfo[kBgWords * bg] = ns > 1 ? first_split_slot(prefix, bg, T) : 0;
+            bginfo[kBgWords * bg + 1] = ns;
+        }
+    }
+    if (k == 0) {
+        int32_t* pg = p.plan_out + prefix_offset_words(G, BG);
+        for (int i = tid; i <= BG; i += nthr) pg[i] = prefix[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) my_slots += __shfl_xor_sync(kFullMask, my_slots, o);
+        if (lane == 0 && my_slots) atomicAdd(total_slots, my_slots);
+    }
+    __syncthreads();
+    if (k == 0 && tid == 0) {
+        int32_t* h = p.plan_out;
+        h[kHdrMagic] = kSchedMagic;
+        h[kHdrG] = G;
+        h[kHdrBG] = BG;
+        h[kHdrHg] = Hg;
+        h[kHdrNG] = NG;
+        h[kHdrSlots] = *total_slots;
+        h[kHdrT] = (int)T;
+        h[kHdrW] = (int)W;
+        h[kHdrBatch] = BG / Hg;
+        h[kHdrMaxBlocks] = mb;
+        h[kHdrShift] = kPageShift;
+        h[kHdrShareHg] = 1;
+        for (int i = kHdrShareHg + 1; i < kHdrWords; ++i) h[i] = 0;
+        if (*bad) atomicOr(p.status, MLA_STATUS_BAD_SEQLEN);
+    }
+}
+
 // ------------------------------------------------------------------ kernels
 template <int NG, class S>
 __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
@@ -1204,53 +1368,80 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Launched as a dependent of the schedule kernel: wait until the plan is
-    // written, then let the combine launch behind this grid.
-    griddep_wait();
-    griddep_launch_dependents();
-    const int32_t* hdr = p.sched;
-    if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
-        __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG ||
-        __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != 1) {
-        if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
-        return;
-    }
-    if constexpr (L::kAlignSlack == 0) {
-        if (smem != smem_raw) {  // no room was reserved to realign the base
-            if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_SMEM_ALIGN);
-            return;
-        }
-    }
-    const int32_t* meta = hdr + kHdrWords + (size_t)blockIdx.x * kMetaWords;
-    const int32_t* bginfo = hdr + bg_offset_words(p.G);
+    MLA_TRACE_K(0);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kBarCount; ++i) {
-            uint32_t count = 1;
-            if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
-                i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged || i == kMaxFull)
-                count = FwdWarps<NG, S>::kSoftmaxThreads;
-            if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
-            if ((i >= kKvEmpty0 && i < kKvEmpty0 + kMaxStages) || i == kPEmpty0 || i == kPEmpty1 ||
-                i == kMmaDone2)
-                count = FwdWarps<NG, S>::kG2Issuers;
-            mbar_init(bar0 + 8 * i, count);
+    int32_t* meta_s = reinterpret_cast<int32_t*>(smem + L::kPlanMetaOff);
+    // A base that could not be realigned (no slack reserved) is reported after
+    // the wait below, with nothing set up.
+    bool misaligned = false;
+    if constexpr (L::kAlignSlack == 0) misaligned = smem != smem_raw;
+    // Setup that reads nothing another grid writes (barriers, TMEM) overlaps
+    // the end of the grid before this one.
+    if (!misaligned) {
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < kBarCount; ++i) {
+                uint32_t count = 1;
+                if (i == kSEmpty0 || i == kSEmpty1 || i == kPFull0 || i == kPFull1 || i == kOEmpty ||
+                    i == kRedFull0 || i == kRedFull1 || i == kSumFull || i == kOutStaged || i == kMaxFull)
+                    count = FwdWarps<NG, S>::kSoftmaxThreads;
+                if (i == kSFull0 || i == kSFull1 || i == kQEmpty || i == kMmaDone) count = G1<NG>::kIssuers;
+                if ((i >= kKvEmpty0 && i < kKvEmpty0 + kMaxStages) || i == kPEmpty0 || i == kPEmpty1 ||
+                    i == kMmaDone2)
+                    count = FwdWarps<NG, S>::kG2Issuers;
+                mbar_init(bar0 + 8 * i, count);
+            }
+            *abort_flag = 0;
+            fence_mbar_init();
         }
-        *abort_flag = 0;
-        fence_mbar_init();
+        if (warp == 1) {
+            tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
+            tmem_relinquish();
+        }
     }
-    if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
-        tmem_relinquish();
-    }
+    // The lengths the plan is built from: into L2 while the grid before this
+    // one may still run (a prefetch returns no data, so a later write to the
+    // lengths still reaches the loads after the wait).
+    if (p.plan_out != nullptr)
+        for (int i = 32 * threadIdx.x; i < p.BG / p.Hg; i += 32 * blockDim.x) prefetch_l2_line(p.seqlens + i);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Launched as a programmatic dependent: wait until the grid before this
+    // one (the schedule kernel, or whatever wrote q and the lengths) is
+    // complete, then let the combine launch behind this grid.
+    griddep_wait();
+    griddep_launch_dependents();
+    MLA_TRACE_K(1);
+    if (misaligned) {
+        if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_SMEM_ALIGN);
+        return;
+    }
     const uint32_t tmem = *tmem_slot;
+    const int32_t* meta;
+    if (p.plan_out != nullptr) {
+        // The plan is built here; the second page stage holds its scratch
+        // until the producer's first copy into it, after the barrier that
+        // ends build_plan_in_cta.
+        build_plan_in_cta(p, NG, reinterpret_cast<int32_t*>(smem + L::kKvOff + L::kStageBytes), meta_s);
+        meta = meta_s;
+    } else {
+        const int32_t* hdr = p.sched;
+        if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
+            __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG ||
+            __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != 1) {
+            if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
+            if (warp == 1) {
+                tc_fence_after();
+                tmem_dealloc(tmem, L::kTmemCols);
+            }
+            return;
+        }
+        meta = hdr + kHdrWords + (size_t)blockIdx.x * kMetaWords;
+    }
     const Ctl ctl{abort_flag, p.status};
+    MLA_TRACE_K(2);
 
     if (warp < FwdWarps<NG, S>::kFirstSoftmax) {
         if constexpr (FwdWarps<NG, S>::kSplitRegs) setmaxnreg_dec<FwdWarps<NG, S>::kRegsIssue>();
@@ -1258,16 +1449,19 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
             if (lane == 0) {
                 prefetch_tensormap(&kv_map);
                 prefetch_tensormap(&q_map);
-                run_producer<NG, S>(&kv_map, &q_map, p, meta, bginfo, smem, ctl);
+                run_producer<NG, S>(&kv_map, &q_map, p, meta, smem, ctl);
             }
         } else if (warp <= G1<NG>::kIssuers) {
-            if (lane == 0) run_gemm1<NG, S>(p, meta, bginfo, smem, tmem, ctl, warp - 1);
+            if (lane == 0) run_gemm1<NG, S>(p, meta, smem, tmem, ctl, warp - 1);
+            MLA_TRACE_K_BY(5, 32);
         } else {
-            if (lane == 0) run_gemm2<NG, S>(p, meta, bginfo, smem, tmem, ctl, warp - FwdWarps<NG, S>::kFirstG2);
+            if (lane == 0) run_gemm2<NG, S>(p, meta, smem, tmem, ctl, warp - FwdWarps<NG, S>::kFirstG2);
+            MLA_TRACE_K_BY(6, (32 * FwdWarps<NG, S>::kFirstG2));
         }
     } else {
         if constexpr (FwdWarps<NG, S>::kSplitRegs) setmaxnreg_inc<FwdWarps<NG, S>::kRegsSoftmax>();
-        run_softmax<NG, S>(p, meta, bginfo, smem, tmem, ctl);
+        run_softmax<NG, S>(p, meta, smem, tmem, ctl);
+        MLA_TRACE_K_BY(7, (32 * FwdWarps<NG, S>::kFirstSoftmax));
     }
     tc_fence_before();
     __syncthreads();
@@ -1275,15 +1469,23 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, L::kTmemCols);
     }
+    MLA_TRACE_K_BY(4, 32);
 }
 
 // LSE-weighted merge of split partials; one CTA per (request-group, column),
-// four output columns d per thread.  After the decode grid completes, the
-// merge is one round of loads: the k partial LSEs are read one per thread and
-// reduced across the block while the first kCombinePre partial rows are
-// already in flight; further rows are read kCombineUnroll at a time.
+// four output columns d per thread.  Up to kCombineFast splits, the merge is
+// one round of loads after the decode grid completes: each thread reads all
+// k partial LSEs and its columns of all k rows and reduces them alone.  With
+// more splits the LSEs are read one per thread and reduced across the block
+// while the first kCombinePre partial rows are already in flight; further
+// rows are read kCombineUnroll at a time.
 constexpr int kCombinePre = 8;
 constexpr int kCombineUnroll = 8;
+// Up to this many splits the merge takes no block reduction.  Measured on
+// B200 (graph-replayed steps): at 4 the 128-head workload's ~8,200 combine
+// CTAs (2-3 splits each) take 8 us less than with block reductions, while
+// raising it to 8 costs the ragged 16-head workload ~4 us.
+constexpr int kCombineFast = 4;
 
 template <int kCombineThreads, bool kMax>
 __device__ __forceinline__ float combine_block_reduce(float v, float* red) {
@@ -1315,8 +1517,10 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     __shared__ float wts[kCombineThreads];
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
-    // The plan may be read before the wait: the decode grid let this grid
-    // start only after its own wait on the grid that wrote the plan.
+    // A plan from the schedule kernel may be read before the wait: the decode
+    // grid let this grid start only after its own wait on the grid that wrote
+    // it.  A plan the decode kernel built itself is complete only after it.
+    if (p.plan_in_decode) griddep_wait();
     const int32_t* hdr = p.sched;
     if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
         __ldg(hdr + kHdrBG) != p.plan_BG || __ldg(hdr + kHdrHg) != p.plan_Hg || __ldg(hdr + kHdrNG) != p.NG ||
@@ -1335,43 +1539,76 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     const int base = __ldg(info + 0);
     const int k = __ldg(info + 1);
     if (k == 1) return;  // unsplit: the decode kernel wrote the final row
-    if (k > 1 && (base < 0 || ((int64_t)base + k) * p.share > p.slots_cap)) {
+    // Slots of the splits: the one-CTA kernels' fixed slots (split_slot), or
+    // the CTA-pair plans' (base + i) * share + group.  In both, split i >= 1
+    // sits at a constant stride from split 1.
+    const bool fixed = p.shift == kPageShift;
+    if (k > 1 && (base < 0 || (fixed ? split_slot(base, k - 1) >= p.slots_cap
+                                     : ((int64_t)base + k) * p.share > p.slots_cap))) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
     const int s = gc / p.heads;
     const int head = gc - s * p.heads;
     const int d0 = threadIdx.x * 4;
-    const size_t slot0 = (size_t)base * p.share + gs;
-    const size_t lstride = (size_t)p.share * p.NG;  // split i -> slot0 + i * share
-    const float* lp = p.lpart + slot0 * p.NG + n;
-    const float* op = p.opart + (slot0 * p.NG + n) * kDv + d0;
-    const size_t ostride = lstride * kDv;
-    griddep_wait();  // the decode grid's partials are complete and visible
+    const size_t slot0 = fixed ? (size_t)base : (size_t)base * p.share + gs;
+    const size_t slot1 = fixed ? (size_t)split_slot(base, 1) : slot0 + p.share;
+    const size_t sstride = fixed ? 2 : (size_t)p.share;
+    auto slot_i = [&](int i) -> size_t { return i == 0 ? slot0 : slot1 + (size_t)(i - 1) * sstride; };
+    const float* lp0 = p.lpart + n;
+    const float* op0 = p.opart + (size_t)n * kDv + d0;
+    auto lse_of = [&](int i) { return __ldg(lp0 + slot_i(i) * p.NG); };
+    auto row_of = [&](int i) { return __ldg(reinterpret_cast<const float4*>(op0 + slot_i(i) * p.NG * kDv)); };
+    MLA_TRACE_STEP_MIN(2);
+    if (!p.plan_in_decode) griddep_wait();  // the decode grid's partials are complete and visible
+    MLA_TRACE_STEP_MIN(3);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lstar = -INFINITY;
-    if (k > 1) {
+    if (k > 1 && k <= kCombineFast) {
+        // Few splits: one round of loads.  Every thread reads the k LSEs (the
+        // same words across the block) next to its four columns of each
+        // partial row, and reduces them itself.
+        float l[kCombineFast];
+        float4 v[kCombineFast];
+#pragma unroll
+        for (int i = 0; i < kCombineFast; ++i)
+            if (i < k) {
+                l[i] = lse_of(i);
+                v[i] = row_of(i);
+            }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kCombineFast; ++i)
+            if (i < k) mx = fmaxf(mx, l[i]);
+        if (mx != -INFINITY) {
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < kCombineFast; ++i)
+                if (i < k) sum += expf(l[i] - mx);
+            lstar = mx + logf(sum);
+#pragma unroll
+            for (int i = 0; i < kCombineFast; ++i)
+                if (i < k) fma4(acc, expf(l[i] - lstar), v[i]);
+        }
+    } else if (k > 1) {
         float4 pre[kCombinePre];
 #pragma unroll
         for (int i = 0; i < kCombinePre; ++i)
-            if (i < k) pre[i] = __ldg(reinterpret_cast<const float4*>(op + (size_t)i * ostride));
-        float own = threadIdx.x < k ? __ldg(lp + (size_t)threadIdx.x * lstride) : -INFINITY;
+            if (i < k) pre[i] = row_of(i);
+        float own = threadIdx.x < k ? lse_of(threadIdx.x) : -INFINITY;
         float mx = own;
-        for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads)
-            mx = fmaxf(mx, __ldg(lp + (size_t)i * lstride));
+        for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads) mx = fmaxf(mx, lse_of(i));
         mx = combine_block_reduce<kCombineThreads, true>(mx, red);
         if (mx != -INFINITY) {  // uniform across the block
             float sum = 0.f;
             for (int i = threadIdx.x; i < k; i += kCombineThreads)
-                sum += expf((i == threadIdx.x ? own : __ldg(lp + (size_t)i * lstride)) - mx);
+                sum += expf((i == threadIdx.x ? own : lse_of(i)) - mx);
             sum = combine_block_reduce<kCombineThreads, false>(sum, red);
             lstar = mx + logf(sum);
             for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
                 const int cn = k - c0 < kCombineThreads ? k - c0 : kCombineThreads;
                 __syncthreads();  // the previous chunk's weights are consumed
-                if (threadIdx.x < cn)
-                    wts[threadIdx.x] =
-                        expf((c0 == 0 ? own : __ldg(lp + (size_t)(c0 + threadIdx.x) * lstride)) - lstar);
+                if (threadIdx.x < cn) wts[threadIdx.x] = expf((c0 == 0 ? own : lse_of(c0 + threadIdx.x)) - lstar);
                 __syncthreads();
                 int i = 0;
                 if (c0 == 0) {
@@ -1383,13 +1620,11 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
                 for (; i + kCombineUnroll <= cn; i += kCombineUnroll) {
                     float4 v[kCombineUnroll];
 #pragma unroll
-                    for (int j = 0; j < kCombineUnroll; ++j)
-                        v[j] = __ldg(reinterpret_cast<const float4*>(op + (size_t)(c0 + i + j) * ostride));
+                    for (int j = 0; j < kCombineUnroll; ++j) v[j] = row_of(c0 + i + j);
 #pragma unroll
                     for (int j = 0; j < kCombineUnroll; ++j) fma4(acc, wts[i + j], v[j]);
                 }
-                for (; i < cn; ++i)
-                    fma4(acc, wts[i], __ldg(reinterpret_cast<const float4*>(op + (size_t)(c0 + i) * ostride)));
+                for (; i < cn; ++i) fma4(acc, wts[i], row_of(c0 + i));
             }
         }
     }
@@ -1405,32 +1640,12 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
         *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) = packed;
     }
     if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
+    MLA_TRACE_STEP_MAX(4);
+#ifdef MLA_TRACE
+    if (threadIdx.x == 0 && bg < 64 && n < 64) g_mla_trace_comb[bg][n] = stamp_timer_ns();
+#endif
 }
 
-// Block-wide inclusive scan of one int per thread (blockDim.x == 1024).
-__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFullMask, v, o);
-        if (lane >= o) v += y;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_tot[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFullMask, w, o);
-            if (lane >= o) w += y;
-        }
-        warp_tot[lane] = w;
-    }
-    __syncthreads();
-    const int r = v + (warp > 0 ? warp_tot[warp - 1] : 0);
-    __syncthreads();
-    return r;
-}
 
 // Builds the persistent-CTA plan on the device (one block of 1024 threads).
 // With use_smem the lengths and the unit prefix live in dynamic shared memory
@@ -1445,6 +1660,7 @@ __global__ void __launch_bounds__(1024)
     __shared__ int bad_len;
     // The decode kernel that follows may launch now; it waits for this grid
     // to complete before it reads the plan.
+    MLA_TRACE_STEP_MIN(0);
     griddep_launch_dependents();
     const int BG = B * Hg;
     int32_t* prefix_g = sched + prefix_offset_words(G, BG);
@@ -1486,19 +1702,19 @@ __global__ void __launch_bounds__(1024)
     }
     __syncthreads();
     const int64_t T = units_per_cta(W, G);
-    for (int k = threadIdx.x; k < G; k += 1024)
-        cta_meta(prefix, BG, W, T, k, seqlens, Hg, max_blocks, shift, meta + (size_t)k * kMetaWords);
+    for (int k = threadIdx.x; k < G; k += 1024) cta_meta(prefix, BG, W, T, k, meta + (size_t)k * kMetaWords);
     __syncthreads();
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     for (int base = 0; base < BG; base += 1024) {
         const int bg = base + threadIdx.x;
         int ns = 0;
-        if (bg < BG) ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, max_blocks, shift), T);
+        if (bg < BG) ns = num_splits_of(prefix, bg, pages_in_prefix(prefix, bg), T);
         const int v = ns > 1 ? ns : 0;
         const int incl = block_inclusive_scan(v, warp_tot);
         if (bg < BG) {
-            bginfo[kBgWords * bg] = carry + incl - v;
+            // one-CTA kernels (64-token units): fixed slots; CTA-pair plans: running count
+            bginfo[kBgWords * bg] = shift != kPageShift ? carry + incl - v : ns > 1 ? first_split_slot(prefix, bg, T) : 0;
             bginfo[kBgWords * bg + 1] = ns;
         }
         __syncthreads();
@@ -1521,6 +1737,7 @@ __global__ void __launch_bounds__(1024)
         sched[kHdrShareHg] = share_hg;
         for (int i = kHdrShareHg + 1; i < kHdrWords; ++i) sched[i] = 0;
     }
+    MLA_TRACE_STEP_MAX(1);
 }
 
 }  // namespace mla

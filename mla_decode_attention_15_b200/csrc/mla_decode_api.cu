@@ -20,9 +20,9 @@ namespace {
 
 using namespace mla;
 
-constexpr int kAbiVersion = 5;
+constexpr int kAbiVersion = 6;
 constexpr int kMaxDevices = 64;
-constexpr int32_t kKnownFlags = MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL | MLA_FLAG_FP32_OUT;
+constexpr int32_t kKnownFlags = MLA_FLAG_NO_COMBINE | MLA_FLAG_TEST_STALL | MLA_FLAG_FP32_OUT | MLA_FLAG_INLINE_PLAN;
 
 int validate_dims(const mla_decode_dims* d) {
     if (d == nullptr) return MLA_ERR_INVALID_ARG;
@@ -317,8 +317,9 @@ struct ColMap {
 
 template <int kDvT>
 int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const void* workspace, void* out,
-                   float* lse, int32_t flags, cudaStream_t stream) {
+                   float* lse, int32_t flags, bool plan_in_decode, cudaStream_t stream) {
     CombineParams c;
+    c.plan_in_decode = plan_in_decode ? 1 : 0;
     c.sched = static_cast<const int32_t*>(schedule);
     c.opart = static_cast<const float*>(workspace);
     c.lpart = c.opart + (size_t)pl.slots * pl.gr.NG * kDvT;
@@ -359,6 +360,31 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
 
 ColMap mla_colmap(const mla_decode_dims* d, const Plan& pl) {
     return ColMap{d->s_q, d->num_heads, pl.gr.NG, 0, d->batch};
+}
+
+// MLA_FLAG_INLINE_PLAN: the one-CTA decode kernel builds the plan itself when
+// its unit prefix fits one page stage; otherwise (CTA-pair kernel, or more
+// request-groups) the call enqueues the schedule kernel before the decode.
+template <class S>
+int inline_plan_cap(int NG) {
+    return NG == 16 ? FwdSmem<16, S>::kInlinePlanMaxBG
+         : NG == 32 ? FwdSmem<32, S>::kInlinePlanMaxBG
+                    : FwdSmem<64, S>::kInlinePlanMaxBG;
+}
+bool plan_in_kernel(int32_t flags, const Plan& pl, bool gqa) {
+    if (!(flags & MLA_FLAG_INLINE_PLAN) || pl.pair) return false;
+    return pl.BG <= (gqa ? inline_plan_cap<ShapeGqa>(pl.gr.NG) : inline_plan_cap<ShapeMla>(pl.gr.NG));
+}
+
+int launch_schedule(const Plan& pl, int batch, int max_blocks, const int32_t* cache_seqlens, void* schedule,
+                    cudaStream_t stream) {
+    // Lengths and unit prefix in shared memory when they fit the default 48 KB.
+    const size_t sh_bytes = ((size_t)batch + pl.BG + 1) * sizeof(int32_t);
+    const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
+    mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, stream>>>(
+        cache_seqlens, static_cast<int32_t*>(schedule), batch, pl.plan_Hg, pl.gr.NG, pl.G, max_blocks, use_smem,
+        pl.shift, pl.share);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 // ---- scratch of the allocation-free entry point ----
@@ -515,13 +541,8 @@ int mla_decode_get_schedule(const mla_decode_dims* dims, const int32_t* cache_se
     int rc = make_plan(dims, &pl);
     if (rc != MLA_OK) return rc;
     if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
-    // Lengths and unit prefix in shared memory when they fit the default 48 KB.
-    const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
-    const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
-    mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
-        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.plan_Hg, pl.gr.NG, pl.G,
-        dims->max_blocks_per_seq, use_smem, pl.shift, pl.share);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return launch_schedule(pl, dims->batch, dims->max_blocks_per_seq, cache_seqlens, schedule,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seqlens, void* schedule_host) {
@@ -546,11 +567,11 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     }
     prefix[BG] = (int32_t)W;
     const int64_t T = units_per_cta(W, G);
-    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, seqlens, Hg, mb, sh, s + kHdrWords + (size_t)k * kMetaWords);
+    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, s + kHdrWords + (size_t)k * kMetaWords);
     int64_t slots = 0;
     for (int bg = 0; bg < BG; ++bg) {
-        const int ns = num_splits_of(prefix, bg, pages_of_bg(seqlens, bg, Hg, mb, sh), T);
-        bginfo[kBgWords * bg] = (int32_t)slots;
+        const int ns = num_splits_of(prefix, bg, pages_in_prefix(prefix, bg), T);
+        bginfo[kBgWords * bg] = pl.pair ? (int32_t)slots : ns > 1 ? first_split_slot(prefix, bg, T) : 0;
         bginfo[kBgWords * bg + 1] = ns;
         if (ns > 1) slots += ns;
     }
@@ -571,7 +592,7 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     return MLA_OK;
 }
 
-int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* workspace, const void* q,
+int mla_decode_fwd(const mla_decode_dims* dims, void* schedule, void* workspace, const void* q,
                    const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
                    float softmax_scale, void* out, float* lse, void* stream) {
     Plan pl;
@@ -587,8 +608,15 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     // Q boxes: the group's rows (one CTA of a pair loads 64 of its 128)
     rc = make_q_map(&qm, q, dims->batch * pl.gr.N, pl.pair ? kPairCols / 2 : pl.gr.NG);
     if (rc != MLA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool in_kernel = plan_in_kernel(dims->flags, pl, false);
+    if ((dims->flags & MLA_FLAG_INLINE_PLAN) && !in_kernel) {
+        rc = launch_schedule(pl, dims->batch, dims->max_blocks_per_seq, cache_seqlens, schedule, st);
+        if (rc != MLA_OK) return rc;
+    }
     FwdParams p;
     p.sched = static_cast<const int32_t*>(schedule);
+    p.plan_out = in_kernel ? static_cast<int32_t*>(schedule) : nullptr;
     p.block_table = block_table;
     p.seqlens = cache_seqlens;
     p.kv = static_cast<const uint8_t*>(kv_cache);
@@ -610,7 +638,6 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     p.run_rows = pl.gr.NG;
     p.run_stride = 0;
     p.kv_groups = 1;
@@ -620,7 +647,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, const void* schedule, void* work
                             : launch_fwd<64, ShapeMla>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
-    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags, st);
+    return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags, in_kernel, st);
 }
 
 int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const void* workspace, void* out,
@@ -631,7 +658,7 @@ int mla_decode_combine(const mla_decode_dims* dims, const void* schedule, const 
     if (!aligned16(schedule) || !aligned16(workspace) || !aligned16(out) || !aligned16(lse))
         return MLA_ERR_INVALID_ARG;
     return launch_combine<kDv>(mla_colmap(dims, pl), pl, schedule, workspace, out, lse, dims->flags,
-                               static_cast<cudaStream_t>(stream));
+                               plan_in_kernel(dims->flags, pl, false), static_cast<cudaStream_t>(stream));
 }
 
 size_t mla_gqa_decode_schedule_bytes(const mla_gqa_dims* dims) {
@@ -652,15 +679,11 @@ int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_s
     int rc = make_plan_gqa(dims, &pl);
     if (rc != MLA_OK) return rc;
     if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
-    const size_t sh_bytes = ((size_t)dims->batch + pl.BG + 1) * sizeof(int32_t);
-    const int use_smem = sh_bytes <= 48 * 1024 ? 1 : 0;
-    mla_decode_schedule_kernel<<<1, 1024, use_smem ? sh_bytes : 0, static_cast<cudaStream_t>(stream)>>>(
-        cache_seqlens, static_cast<int32_t*>(schedule), dims->batch, pl.plan_Hg, pl.gr.NG, pl.G,
-        dims->max_blocks_per_seq, use_smem, pl.shift, pl.share);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return launch_schedule(pl, dims->batch, dims->max_blocks_per_seq, cache_seqlens, schedule,
+                           static_cast<cudaStream_t>(stream));
 }
 
-int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* workspace, const void* q,
+int mla_gqa_decode_fwd(const mla_gqa_dims* dims, void* schedule, void* workspace, const void* q,
                        const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
                        float softmax_scale, void* out, float* lse, void* stream) {
     Plan pl;
@@ -675,8 +698,15 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
     if (rc != MLA_OK) return rc;
     rc = make_q_map(&qm, q, dims->batch * pl.gr.N, kGqaHeadsPerGroup, ShapeGqa::kDqk);
     if (rc != MLA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool in_kernel = plan_in_kernel(dims->flags, pl, true);
+    if ((dims->flags & MLA_FLAG_INLINE_PLAN) && !in_kernel) {
+        rc = launch_schedule(pl, dims->batch, dims->max_blocks_per_seq, cache_seqlens, schedule, st);
+        if (rc != MLA_OK) return rc;
+    }
     FwdParams p;
     p.sched = static_cast<const int32_t*>(schedule);
+    p.plan_out = in_kernel ? static_cast<int32_t*>(schedule) : nullptr;
     p.block_table = block_table;
     p.seqlens = cache_seqlens;
     p.kv = static_cast<const uint8_t*>(kv_cache);
@@ -701,12 +731,11 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, const void* schedule, void* wor
     p.run_rows = kGqaHeadsPerGroup;  // one run of 16 heads per new token
     p.run_stride = dims->num_q_heads;
     p.kv_groups = dims->num_kv_groups;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = pl.gr.NG == 16 ? launch_fwd<16, ShapeGqa>(pl, p, kvm, qm, st) : launch_fwd<32, ShapeGqa>(pl, p, kvm, qm, st);
     if (rc != MLA_OK) return rc;
     if (dims->flags & MLA_FLAG_NO_COMBINE) return MLA_OK;
     return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads, dims->batch},
-                                         pl, schedule, workspace, out, lse, dims->flags, st);
+                                         pl, schedule, workspace, out, lse, dims->flags, in_kernel, st);
 }
 
 int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const void* workspace, void* out,
@@ -718,7 +747,7 @@ int mla_gqa_decode_combine(const mla_gqa_dims* dims, const void* schedule, const
         return MLA_ERR_INVALID_ARG;
     return launch_combine<ShapeGqa::kDv>(ColMap{dims->s_q, dims->num_q_heads, kGqaHeadsPerGroup, dims->num_q_heads, dims->batch},
                                          pl, schedule, workspace, out, lse, dims->flags,
-                                         static_cast<cudaStream_t>(stream));
+                                         plan_in_kernel(dims->flags, pl, true), static_cast<cudaStream_t>(stream));
 }
 
 #ifdef MLA_TRACE
@@ -728,6 +757,29 @@ int mla_decode_trace_fetch(void* events_host, size_t events_bytes, void* counts_
     if (events_bytes != sizeof(g_mla_trace) || counts_bytes != sizeof(g_mla_trace_count)) return MLA_ERR_INVALID_ARG;
     if (cudaMemcpyFromSymbol(events_host, g_mla_trace, events_bytes) != cudaSuccess ||
         cudaMemcpyFromSymbol(counts_host, g_mla_trace_count, counts_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+// Copies the combine CTAs' exit stamps.
+int mla_decode_trace_fetch_comb(void* host, size_t bytes) {
+    if (bytes != sizeof(g_mla_trace_comb)) return MLA_ERR_INVALID_ARG;
+    if (cudaMemcpyFromSymbol(host, g_mla_trace_comb, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+// Copies the kernel-level stamps (decode CTAs, then the step's five) and
+// resets the step stamps for the next call.
+int mla_decode_trace_fetch_k(void* k_host, size_t k_bytes, void* step_host, size_t step_bytes) {
+    if (k_bytes != sizeof(g_mla_trace_k) || step_bytes != sizeof(g_mla_trace_step)) return MLA_ERR_INVALID_ARG;
+    unsigned long long init[8];
+    for (int i = 0; i < 8; ++i) init[i] = (i == 1 || i == 4) ? 0ull : ~0ull;
+    if (cudaMemcpyFromSymbol(k_host, g_mla_trace_k, k_bytes) != cudaSuccess ||
+        cudaMemcpyFromSymbol(step_host, g_mla_trace_step, step_bytes) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_mla_trace_step, init, sizeof(init)) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }

@@ -59,7 +59,7 @@ enum HdrField {
 };
 constexpr int kMetaWords = 8;  // per CTA: begin_bg, begin_page, end_bg, end_page, first_split
 enum MetaField { kMetaBeginBg = 0, kMetaBeginPage = 1, kMetaEndBg = 2, kMetaEndPage = 3, kMetaFirstSplit = 4 };
-constexpr int kBgWords = 2;  // per bg: slot_base, num_splits
+constexpr int kBgWords = 2;  // per bg: slot of split 0 (or the pair plans' slot base), num_splits
 
 __host__ __device__ inline int64_t meta_offset_words() { return kHdrWords; }
 __host__ __device__ inline int64_t bg_offset_words(int G) { return kHdrWords + (int64_t)kMetaWords * G; }
@@ -128,23 +128,24 @@ __host__ __device__ inline int find_bg(const int32_t* prefix, int BG, int64_t u)
     return lo;
 }
 
-// Blocks of request-group bg under the clamp every kernel applies.
-__host__ __device__ inline int pages_of_bg(const int32_t* seqlens, int bg, int Hg, int max_blocks,
-                                           int shift = kPageShift) {
-    return blocks_of(clamp_seqlen(seqlens[bg / Hg], max_blocks), shift);
+// Blocks of request-group bg (of its length clamped to the block table),
+// read back from the unit prefix: its units are P + kItemOverhead, or 0 when
+// P == 0.  No access to the lengths.
+__host__ __device__ inline int pages_in_prefix(const int32_t* prefix, int bg) {
+    const int units = prefix[bg + 1] - prefix[bg];
+    return units > 0 ? units - kItemOverhead : 0;
 }
 
 // (bg, page) position of unit u; u >= W maps to (BG, 0).
-__host__ __device__ inline void locate_unit(const int32_t* prefix, int BG, int64_t W, int64_t u,
-                                            const int32_t* seqlens, int Hg, int max_blocks, int shift,
-                                            int* bg_out, int* page_out) {
+__host__ __device__ inline void locate_unit(const int32_t* prefix, int BG, int64_t W, int64_t u, int* bg_out,
+                                            int* page_out) {
     if (u >= W) {
         *bg_out = BG;
         *page_out = 0;
         return;
     }
     int bg = find_bg(prefix, BG, u);
-    int P = pages_of_bg(seqlens, bg, Hg, max_blocks, shift);
+    int P = pages_in_prefix(prefix, bg);
     int64_t p = u - (int64_t)prefix[bg] - kItemOverhead;
     if (p < 0) p = 0;
     if (p > P) p = P;
@@ -166,18 +167,17 @@ __host__ __device__ inline int num_splits_of(const int32_t* prefix, int bg, int 
 
 // Work range of CTA k: units [k*T, min((k+1)*T, W)).
 __host__ __device__ inline void cta_meta(const int32_t* prefix, int BG, int64_t W, int64_t T, int k,
-                                         const int32_t* seqlens, int Hg, int max_blocks, int shift,
                                          int32_t* meta) {
     int64_t u0 = (int64_t)k * T;
     int64_t u1 = u0 + T;
     if (u0 > W) u0 = W;
     if (u1 > W) u1 = W;
     int bb, bp, eb, ep;
-    locate_unit(prefix, BG, W, u0, seqlens, Hg, max_blocks, shift, &bb, &bp);
-    locate_unit(prefix, BG, W, u1, seqlens, Hg, max_blocks, shift, &eb, &ep);
+    locate_unit(prefix, BG, W, u0, &bb, &bp);
+    locate_unit(prefix, BG, W, u1, &eb, &ep);
     int first_split = 0;
     if (bb < BG) {
-        int P = pages_of_bg(seqlens, bb, Hg, max_blocks, shift);
+        int P = pages_in_prefix(prefix, bb);
         if (P > 0) {
             first_split = k - first_cta_of(prefix, bb, T);
             if (first_split < 0) first_split = 0;
@@ -193,5 +193,23 @@ __host__ __device__ inline void cta_meta(const int32_t* prefix, int BG, int64_t 
 
 // Upper bound of partial slots: every CTA has at most two partial items.
 __host__ __device__ inline int64_t max_slots(int G) { return 2 * (int64_t)G; }
+
+// ---- partial-output slots of the one-CTA kernels ----
+// CTA k writes the partial of its first work item to slot 2k and that of its
+// last item (when that is another, split request-group) to slot 2k + 1, so a
+// CTA places its partials without knowing any other CTA's split count.  A
+// request-group whose first page is on CTA c0 and that is split ns ways then
+// keeps split i >= 1 in slot 2 (c0 + i), since it opens each later CTA's
+// range, and split 0 in slot 2 c0 if it also opens c0's range, else 2 c0 + 1.
+// (CTA-pair plans, whose head groups share each range, number their slots
+// (base + split) * groups + group, with base a running count over requests.)
+__host__ __device__ inline int cta_slot(int k, bool first_item) { return 2 * k + (first_item ? 0 : 1); }
+__host__ __device__ inline int first_split_slot(const int32_t* prefix, int bg, int64_t T) {
+    const int c0 = first_cta_of(prefix, bg, T);
+    return cta_slot(c0, (int64_t)c0 * T >= (int64_t)prefix[bg]);
+}
+__host__ __device__ inline int64_t split_slot(int slot0, int i) {
+    return i == 0 ? (int64_t)slot0 : 2 * ((int64_t)(slot0 >> 1) + i);
+}
 
 }  // namespace mla

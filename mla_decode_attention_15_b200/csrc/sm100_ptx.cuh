@@ -20,6 +20,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+// For timeline stamps: the memory clobber keeps the read in program order
+// with the surrounding memory operations and barriers (without it the
+// compiler may hoist it above a __syncthreads).  Bounded waits use the plain
+// read above, which leaves their loops free to keep values in registers.
+__device__ __forceinline__ uint64_t stamp_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) :: "memory");
+    return t;
+}
+
+// Prefetch of one global line into L2 (no data returned; safe while another
+// grid may still write the line, since the later real load reads L2).
+__device__ __forceinline__ void prefetch_l2_line(const void* gptr) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(gptr) : "memory");
+}
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -85,7 +85,11 @@ def read_plan(buf: np.ndarray, G: int, BG: int):
 def walk_plan(meta, bginfo, seqlens, Hg, max_blocks, shift=6):
     """Items each work range holds, exactly as the decode kernels walk it:
     list per range of (bg, p0, p1, unsplit, slot), in units of 2^shift tokens
-    (64-token pages, or the CTA-pair kernel's 128-token steps)."""
+    (64-token pages, or the CTA-pair kernel's 128-token steps).  The one-CTA
+    kernels (64-token units) put the partial of range k's first item in slot
+    2k and that of its last in 2k + 1; the CTA-pair plans count slots per
+    request (slot base of the request + split index; the head group offset is
+    left out here)."""
     BG = bginfo.shape[0]
     unit = 1 << shift
     out = []
@@ -104,7 +108,12 @@ def walk_plan(meta, bginfo, seqlens, Hg, max_blocks, shift=6):
             if p0 >= p1:
                 continue
             unsplit = p0 == 0 and p1 == P
-            slot = -1 if unsplit else int(bginfo[cur, 0]) + (fs if cur == bb else 0)
+            if unsplit:
+                slot = -1
+            elif shift == 6:
+                slot = 2 * k + (0 if cur == bb else 1)
+            else:
+                slot = int(bginfo[cur, 0]) + (fs if cur == bb else 0)
             items.append((cur, p0, p1, unsplit, slot))
         out.append(items)
     return out

@@ -43,7 +43,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_version_and_strerror(lib):
-    assert bd.mla_decode_version() == 5
+    assert bd.mla_decode_version() == 6
     for code in (0, -1, -2, -3, -4):
         assert bd.mla_decode_strerror(code)
     assert "unknown" in bd.mla_decode_strerror(-99)

@@ -65,10 +65,20 @@ def check_invariants(pl):
         if ns == 1:
             assert pieces[bg][0][3]  # unsplit, written directly
         if ns > 1:
-            slots = sorted(pc[4] for pc in pieces[bg])
+            slots = [pc[4] for pc in pieces[bg]]  # in split order (ascending range)
             base = int(bginfo[bg, 0])
-            assert slots == list(range(base, base + ns))
+            if pl["shift"] == 6:
+                # the slots the combine reads (split_slot) are the ones the pieces were written to
+                expect = [base if i == 0 else 2 * ((base >> 1) + i) for i in range(ns)]
+                assert slots == expect, (bg, slots, expect)
+                assert pieces[bg][0][0] == base >> 1  # split 0 sits on the group's first range
+            else:
+                assert sorted(slots) == list(range(base, base + ns))
             assert not any(pc[3] for pc in pieces[bg])
+    used = [pc[4] for bg in range(BG) for pc in pieces[bg] if not pc[3]]
+    assert len(used) == len(set(used)), "two partials share a slot"
+    if pl["shift"] == 6:
+        assert all(0 <= x < 2 * G for x in used)
     total_slots = sum(int(bginfo[bg, 1]) for bg in range(BG) if bginfo[bg, 1] > 1)
     assert total_slots == int(hdr[5]) <= 2 * G
     return items
