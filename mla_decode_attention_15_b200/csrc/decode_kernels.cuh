@@ -254,7 +254,11 @@ struct FwdParams {
     float* lpart;  // [slots][NG]
     int32_t* status;
     int s_q, heads, N, num_blocks, max_blocks, causal;
-    int G, BG, Hg, slots_cap;
+    int G, BG, Hg, slots_cap;  // plan ranges, plan rows, head groups per plan row, partial slots
+    // One-CTA kernels: CTAs walking each plan range side by side, one per
+    // head group (1: none; >1: the plan has one row per request and CTA c
+    // walks range c / share for head group c % share).
+    int share;
     int out_f32;       // MLA_FLAG_FP32_OUT: final rows are written as fp32
     float scale_log2;  // softmax_scale * log2(e)
     int test_stall;    // MLA_FLAG_TEST_STALL: leave the first page unloaded
@@ -407,15 +411,18 @@ struct Item {
 
 struct WorkIter {
     int bg, begin_bg, begin_page, end_bg, end_page;
+    int range, group;  // plan range of this CTA; its head group when ranges are shared
 
     // meta: this CTA's row of the plan, in the schedule buffer or (plan built
     // by the kernel itself) in shared memory.
-    __device__ void init(const int32_t* meta) {
+    __device__ void init(const int32_t* meta, const FwdParams& p) {
         begin_bg = meta[kMetaBeginBg];
         begin_page = meta[kMetaBeginPage];
         end_bg = meta[kMetaEndBg];
         end_page = meta[kMetaEndPage];
         bg = begin_bg;
+        range = blockIdx.x / p.share;
+        group = blockIdx.x - range * p.share;
     }
 
     __device__ bool next(const FwdParams& p, Item& it) {
@@ -430,7 +437,7 @@ struct WorkIter {
             if (p0 >= p1) continue;
             it.bg = cur;
             it.b = b;
-            it.g = cur - b * p.Hg;
+            it.g = p.share > 1 ? group : cur - b * p.Hg;
             it.p0 = p0;
             it.p1 = p1;
             it.P = P;
@@ -438,8 +445,9 @@ struct WorkIter {
             it.unsplit = (p0 == 0 && p1 == P);
             it.slot = -1;
             if (!it.unsplit) {
-                // first item: slot 2k; last item: slot 2k + 1 (see cta_slot)
-                const int s = cta_slot(blockIdx.x, cur == begin_bg);
+                // first item of the range: slot 2k; last item: slot 2k + 1 (see
+                // cta_slot), times the groups sharing the range, plus this group
+                const int s = cta_slot(range, cur == begin_bg) * p.share + group;
                 it.slot = s < p.slots_cap ? s : -1;
             }
             return true;
@@ -560,7 +568,7 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     const uint64_t policy = p.Hg > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
     WorkIter it;
-    it.init(meta);
+    it.init(meta, p);
     Item item;
     uint32_t kv_it = 0, q_it = 0;
     uint32_t issued[kMaxStages] = {};  // pages loaded per stage (for the abort drain)
@@ -646,7 +654,7 @@ __device__ void run_gemm1(const FwdParams& p, const int32_t* meta,
     const uint32_t q_s = smem_addr(smem + L::kQOff);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     WorkIter it;
-    it.init(meta);
+    it.init(meta, p);
     Item item;
     uint32_t s_it = 0, q_it = 0;
     bool ok = true;
@@ -715,7 +723,7 @@ __device__ void run_gemm2(const FwdParams& p, const int32_t* meta,
     const uint32_t p_s = kv_s + L::kPInStage;  // P^T of stage 0
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     WorkIter it;
-    it.init(meta);
+    it.init(meta, p);
     Item item;
     uint32_t s_it = 0, item_it = 0;
     bool ok = true;
@@ -812,7 +820,7 @@ __device__ void run_softmax(const FwdParams& p, const int32_t* meta,
 #endif
 
     WorkIter it;
-    it.init(meta);
+    it.init(meta, p);
     Item item;
     uint32_t s_it = 0, item_it = 0, out_it = 0, max_it = 0;
     bool ok = true;
@@ -1267,7 +1275,10 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
 // end, after which the scratch stage is free.
 __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, int32_t* plan_s) {
     const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
-    const int k = blockIdx.x, G = gridDim.x, BG = p.BG, Hg = p.Hg, mb = p.max_blocks;
+    // With shared ranges every CTA of range k computes the same plan; the one
+    // of group 0 writes the range's share of it.
+    const int k = blockIdx.x / p.share, G = gridDim.x / p.share, BG = p.BG, Hg = p.Hg, mb = p.max_blocks;
+    const bool writer = blockIdx.x % p.share == 0;
     int32_t* prefix = scratch;
     int32_t* warp_tot = scratch + BG + 1;
     int32_t* meta_s = plan_s;
@@ -1315,7 +1326,8 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
     if (tid == 0) {
         cta_meta(prefix, BG, W, T, k, meta_s);
         int32_t* row = p.plan_out + kHdrWords + (size_t)k * kMetaWords;
-        for (int i = 0; i < kMetaWords; ++i) row[i] = meta_s[i];
+        if (writer)
+            for (int i = 0; i < kMetaWords; ++i) row[i] = meta_s[i];
     }
     int32_t* bginfo = p.plan_out + bg_offset_words(G);
     int my_slots = 0;
@@ -1325,12 +1337,12 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
         if (ns > 1) my_slots += ns;
         int owner = P > 0 ? first_cta_of(prefix, bg, T) : 0;
         if (owner > G - 1) owner = G - 1;
-        if (owner == k) {
+        if (owner == k && writer) {
             bginfo[kBgWords * bg] = ns > 1 ? first_split_slot(prefix, bg, T) : 0;
             bginfo[kBgWords * bg + 1] = ns;
         }
     }
-    if (k == 0) {
+    if (blockIdx.x == 0) {
         int32_t* pg = p.plan_out + prefix_offset_words(G, BG);
         for (int i = tid; i <= BG; i += nthr) pg[i] = prefix[i];
 #pragma unroll
@@ -1338,7 +1350,7 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
         if (lane == 0 && my_slots) atomicAdd(total_slots, my_slots);
     }
     __syncthreads();
-    if (k == 0 && tid == 0) {
+    if (blockIdx.x == 0 && tid == 0) {
         int32_t* h = p.plan_out;
         h[kHdrMagic] = kSchedMagic;
         h[kHdrG] = G;
@@ -1351,7 +1363,7 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
         h[kHdrBatch] = BG / Hg;
         h[kHdrMaxBlocks] = mb;
         h[kHdrShift] = kPageShift;
-        h[kHdrShareHg] = 1;
+        h[kHdrShareHg] = p.share;
         for (int i = kHdrShareHg + 1; i < kHdrWords; ++i) h[i] = 0;
         if (*bad) atomicOr(p.status, MLA_STATUS_BAD_SEQLEN);
     }
@@ -1430,7 +1442,7 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
         const int32_t* hdr = p.sched;
         if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
             __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG ||
-            __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != 1) {
+            __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != p.share) {
             if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
             if (warp == 1) {
                 tc_fence_after();
@@ -1438,7 +1450,7 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
             }
             return;
         }
-        meta = hdr + kHdrWords + (size_t)blockIdx.x * kMetaWords;
+        meta = hdr + kHdrWords + (size_t)(blockIdx.x / p.share) * kMetaWords;
     }
     const Ctl ctl{abort_flag, p.status};
     MLA_TRACE_K(2);
@@ -1539,11 +1551,12 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     const int base = __ldg(info + 0);
     const int k = __ldg(info + 1);
     if (k == 1) return;  // unsplit: the decode kernel wrote the final row
-    // Slots of the splits: the one-CTA kernels' fixed slots (split_slot), or
-    // the CTA-pair plans' (base + i) * share + group.  In both, split i >= 1
-    // sits at a constant stride from split 1.
+    // Slots of the splits: the one-CTA kernels' fixed slots (split_slot, times
+    // the groups sharing a range, plus the group), or the CTA-pair plans'
+    // (base + i) * share + group.  In both, split i >= 1 sits at a constant
+    // stride from split 1.
     const bool fixed = p.shift == kPageShift;
-    if (k > 1 && (base < 0 || (fixed ? split_slot(base, k - 1) >= p.slots_cap
+    if (k > 1 && (base < 0 || (fixed ? split_slot(base, k - 1) * p.share + gs >= p.slots_cap
                                      : ((int64_t)base + k) * p.share > p.slots_cap))) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
@@ -1551,9 +1564,9 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     const int s = gc / p.heads;
     const int head = gc - s * p.heads;
     const int d0 = threadIdx.x * 4;
-    const size_t slot0 = fixed ? (size_t)base : (size_t)base * p.share + gs;
-    const size_t slot1 = fixed ? (size_t)split_slot(base, 1) : slot0 + p.share;
-    const size_t sstride = fixed ? 2 : (size_t)p.share;
+    const size_t slot0 = (size_t)base * p.share + gs;
+    const size_t slot1 = fixed ? (size_t)split_slot(base, 1) * p.share + gs : slot0 + p.share;
+    const size_t sstride = fixed ? 2 * (size_t)p.share : (size_t)p.share;
     auto slot_i = [&](int i) -> size_t { return i == 0 ? slot0 : slot1 + (size_t)(i - 1) * sstride; };
     const float* lp0 = p.lpart + n;
     const float* op0 = p.opart + (size_t)n * kDv + d0;

@@ -174,13 +174,25 @@ int make_plan_gqa(const mla_gqa_dims* d, Plan* pl) {
     pl->gr.N = d->num_q_heads * d->s_q;
     pl->gr.NG = kGqaHeadsPerGroup * d->s_q;
     pl->gr.Hg = d->num_kv_groups;
-    pl->BG = d->batch * d->num_kv_groups;
-    pl->plan_Hg = pl->gr.Hg;
     pl->shift = kPageShift;
-    pl->share = 1;
-    pl->ctas = pl->G;
     pl->pair = false;
-    pl->slots = max_slots(pl->G);
+    const int sms = pl->G;
+    if (d->num_kv_groups > 1 && sms / d->num_kv_groups >= 1) {
+        // Shared ranges: the plan has one row per request, and each range is
+        // walked by the request's KV groups side by side, one CTA per group,
+        // so that the groups read each page's shared RoPE box at about the
+        // same time and all but the first read hit L2.
+        pl->G = sms / d->num_kv_groups;
+        pl->BG = d->batch;
+        pl->plan_Hg = 1;
+        pl->share = d->num_kv_groups;
+    } else {
+        pl->BG = d->batch * d->num_kv_groups;
+        pl->plan_Hg = pl->gr.Hg;
+        pl->share = 1;
+    }
+    pl->ctas = pl->G * pl->share;
+    pl->slots = max_slots(pl->G) * pl->share;
     return MLA_OK;
 }
 
@@ -635,6 +647,7 @@ int mla_decode_fwd(const mla_decode_dims* dims, void* schedule, void* workspace,
     p.G = pl.G;
     p.BG = pl.BG;
     p.Hg = pl.pair ? pl.share : pl.gr.Hg;  // pair kernel: head groups walking each range
+    p.share = 1;
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;
@@ -724,7 +737,8 @@ int mla_gqa_decode_fwd(const mla_gqa_dims* dims, void* schedule, void* workspace
     p.causal = dims->causal;
     p.G = pl.G;
     p.BG = pl.BG;
-    p.Hg = pl.gr.Hg;
+    p.Hg = pl.plan_Hg;
+    p.share = pl.share;
     p.slots_cap = (int)pl.slots;
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.test_stall = (dims->flags & MLA_FLAG_TEST_STALL) ? 1 : 0;

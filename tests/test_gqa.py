@@ -19,10 +19,17 @@ def lib():
 
 
 def test_gqa_sizes_and_rejections(lib):
+    # 8 KV groups share each work range (one CTA per group): 148 // 8 = 18 ranges,
+    # one plan row per request, 2 partial slots per range and group
     d = bd.make_gqa_dims(16, 2, 8, 1000, 64, True, 148)
-    BG = 16 * 8
-    assert bd.mla_gqa_decode_schedule_bytes(d) == 4 * (16 + 8 * 148 + 3 * BG + 1)
-    assert bd.mla_gqa_decode_workspace_bytes(d) == 2 * 148 * 32 * (128 + 1) * 4
+    G, BG = 148 // 8, 16
+    assert bd.mla_gqa_decode_schedule_bytes(d) == 4 * (16 + 8 * G + 3 * BG + 1)
+    assert bd.mla_gqa_decode_workspace_bytes(d) == 2 * G * 8 * 32 * (128 + 1) * 4
+    # one KV group, or too few SMs for one range per group: one plan row per request-group
+    d1 = bd.make_gqa_dims(16, 2, 1, 1000, 64, True, 148)
+    assert bd.mla_gqa_decode_schedule_bytes(d1) == 4 * (16 + 8 * 148 + 3 * 16 + 1)
+    d7 = bd.make_gqa_dims(16, 2, 8, 1000, 64, True, 7)
+    assert bd.mla_gqa_decode_schedule_bytes(d7) == 4 * (16 + 8 * 7 + 3 * 128 + 1)
     for change, code in [(dict(num_q_heads=24), bd.MLA_ERR_UNSUPPORTED), (dict(s_q=3), bd.MLA_ERR_UNSUPPORTED),
                          (dict(d_head=64), bd.MLA_ERR_UNSUPPORTED), (dict(page_size=32), bd.MLA_ERR_UNSUPPORTED),
                          (dict(batch=0), bd.MLA_ERR_INVALID_ARG), (dict(flags=0x100), bd.MLA_ERR_INVALID_ARG),

@@ -126,8 +126,12 @@ def test_plan_at_the_shared_memory_limit(dev):
 
 
 def test_gqa_matches_two_launch_path(dev):
-    for B, groups, lens in ((6, 8, [1, 64, 65, 1000, 0, 3000]), (1300, 8, None)):
-        if lens is None:  # 10,400 request-groups: more than the kernel plans itself
+    """8 KV groups walk shared ranges (one plan row per request: 6 and 1,300
+    rows); one KV group with 10,200 requests has more plan rows than the
+    kernel builds in one 40 KB page stage, so the call runs the schedule
+    kernel first."""
+    for B, groups, lens in ((6, 8, [1, 64, 65, 1000, 0, 3000]), (1300, 8, None), (10200, 1, None)):
+        if lens is None:
             lens = [1 + (i * 53) % 130 for i in range(B)]
         d = workloads.build_gqa(B, 2, groups, ("list", lens), seed=B, causal=True, pool_device="cuda")
         g = to_dev(d, dev)
