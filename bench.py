@@ -874,6 +874,68 @@ def run_gqa_bench(args):
     return 0
 
 
+def run_composed(args, dev, stream):
+    """One absorbed-MLA layer at the bs16 x 4K x 16-head decode batch (16
+    tokens x 16 heads): mla_absorb_q -> mla_decode_fwd (inline plan, combine)
+    -> mla_absorb_o, each a programmatic dependent of the kernel before it,
+    against mla_decode_fwd alone on the same inputs.  Both graph-replayed
+    with L2 flushed before each replay (the layer's 4 MB of weights then come
+    from HBM, as they do when a model's layers run in turn); medians."""
+    w = workloads.WORKLOADS["b16_l4096_h16"]
+    d = workloads.make_inputs(w)
+    q, kv = d["q"].to(dev), d["kv_cache"].to(dev)
+    bt, sl = d["block_table"].to(dev), d["cache_seqlens"].to(dev)
+    B, s_q, h = w.batch, w.s_q, w.heads
+    x = workloads.build_absorb(B * s_q, h, seed=1400)
+    q_in = x["q_in"].view(B, s_q, h, 192).to(dev)
+    w_uk, w_uv = x["w_uk"].to(dev), x["w_uv"].to(dev)
+    dims = bd.make_dims(B, s_q, h, kv.shape[0], bt.shape[1], w.causal, 0, bd.MLA_FLAG_INLINE_PLAN)
+    sched = torch.empty(bd.mla_decode_schedule_bytes(dims), dtype=torch.uint8, device=dev)
+    ws = torch.empty(bd.mla_decode_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, s_q, h, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, h, s_q, dtype=torch.float32, device=dev)
+    q_lat = torch.empty(B, s_q, h, 576, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(B, s_q, h, 128, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    adims = bd.make_absorb_dims(B * s_q, h)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    bd.mla_decode_get_schedule(dims, sl, sched, stream)
+
+    def decode_only(st):
+        bd.mla_decode_fwd(dims, sched, ws, q, kv, bt, sl, d["softmax_scale"], out, lse, st)
+
+    def layer(st):
+        bd.mla_absorb_q(adims, q_in, w_uk, q_lat, status, st)
+        bd.mla_decode_fwd(dims, sched, ws, q_lat, kv, bt, sl, d["softmax_scale"], out, lse, st)
+        bd.mla_absorb_o(adims, out, w_uv, y, status, st)
+
+    res = {}
+    for tag, fn in (("decode_us", decode_only), ("layer_us", layer)):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            fn(cap)
+            with torch.cuda.graph(g, stream=cap):
+                fn(cap)
+        stream.wait_stream(cap)
+        n = max(3, args.warmup) + args.steps
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(n):
+            flush_l2(flush, i)
+            evs[i][0].record(stream)
+            g.replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        res[tag] = statistics.median(a.elapsed_time(b) * 1e3 for a, b in evs[max(3, args.warmup):])
+        del g
+    assert int(status.max()) == 0 and bd.mla_decode_get_status(sched) == 0
+    res["projections_us"] = res["layer_us"] - res["decode_us"]
+    res["config"] = ("b16_l4096_h16 decode with its 16 tokens x 16 heads projected: W_UK [16,128,512], "
+                     "W_UV [16,512,128]; L2 flushed before each replay")
+    return res
+
+
 def run_absorb_bench(args):
     """The absorbed projections around the decode (GQLA summary, "Caminho
     MQA-Absorvido") at the decode batches of the two measured configurations.
@@ -957,6 +1019,7 @@ def run_absorb_bench(args):
                      "peak_kind": peak_kind + " (copy bandwidth, burst)", "traffic": traffic,
                      "traffic_note": "DRAM bytes of one absorb_q + one absorb_o launch (ncu, 1 pass)"},
         "cases": cases, "gpu_launches": 2 * layers * args.steps,
+        "composed_layer": run_composed(args, dev, stream),
     }
     print(json.dumps(line), flush=True)
     return 0

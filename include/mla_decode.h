@@ -96,7 +96,12 @@ extern "C" {
  * decode kernel.  The status word is not cleared by these calls: call
  * mla_decode_get_schedule once on a new buffer to clear it, after which it
  * collects the faults of every later call until the next
- * mla_decode_get_schedule.  Pass the same flags to mla_decode_combine. */
+ * mla_decode_get_schedule.  Pass the same flags to mla_decode_combine.
+ * The decode kernel is a programmatic dependent of the kernel before it on
+ * the stream and reads cache_seqlens before it waits for that kernel's end:
+ * the lengths must be final when that kernel lets its dependents start.
+ * Kernels that do not use programmatic launch, and this library's own
+ * kernels, always satisfy this. */
 #define MLA_FLAG_INLINE_PLAN 0x8
 
 typedef struct mla_decode_dims {

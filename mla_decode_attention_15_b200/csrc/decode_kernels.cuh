@@ -334,7 +334,7 @@ struct FwdSmem {
     static constexpr int kBarOff = kVoteOff + 2 * 8 * 4;
     static constexpr int kNumBars = 32;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag
-    static constexpr int kPlanMetaOff = kMiscOff + 16;         // this CTA's plan row (+2 words), when built in the kernel
+    static constexpr int kPlanMetaOff = kMiscOff + 16;         // this CTA's plan row + 4 words, when built in the kernel
     static constexpr int kBytes = kPlanMetaOff + (kMetaWords + 8) * 4;
     // largest plan (request-groups) the kernel builds itself: prefix + scan state in one stage
     static constexpr int kInlinePlanMaxBG = kStageBytes / 4 - 48;  // prefix (BG + 1) + 32 warp totals
@@ -558,15 +558,44 @@ __device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const float (&v)
 }
 
 // ------------------------------------------------------------------ roles
+// L2 policy of the page loads: pages that other CTAs read too (the head
+// groups of a plan row) stay normal, the rest are evicted first.  (Marking the
+// pages of shared GQA ranges normal too measured no better: 0.827 against
+// 0.844 of the copy bandwidth.)
+__device__ __forceinline__ uint64_t page_policy(const FwdParams& p) {
+    return p.Hg > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
+}
+
+// Page j of item into stage st: its block-table entry, then the stage's boxes
+// on the stage's "landed" barrier.
+template <int NG, class S>
+__device__ __forceinline__ void issue_page(const CUtensorMap* kv_map, const FwdParams& p, const Item& item, int j,
+                                           int st, uint8_t* smem, uint64_t policy) {
+    using L = FwdSmem<NG, S>;
+    const int32_t* bt = p.block_table + (size_t)item.b * p.max_blocks;
+    int phys = __ldg(bt + j);
+    if ((unsigned)phys >= (unsigned)p.num_blocks) {
+        atomicOr(p.status, MLA_STATUS_BAD_BLOCK_TABLE);
+        phys = 0;
+    }
+    const uint32_t full = smem_addr(smem + L::kBarOff) + 8 * (kKvFull0 + st);
+    mbar_arrive_expect_tx(full, L::kStageBytes);
+    const uint32_t dst = smem_addr(smem + L::kKvOff) + st * L::kStageBytes;
+#pragma unroll
+    for (int c = 0; c < L::kBoxes; ++c)
+        tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, S::col(c, item.g, p.kv_groups), 0, phys, policy);
+}
+
+// first_page_issued: the kernel already issued the first page of the first
+// item into stage 0, before its wait on the previous grid.
 template <int NG, class S>
 __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map,
                              const FwdParams& p, const int32_t* meta,
-                             uint8_t* smem, const Ctl& ctl) {
+                             uint8_t* smem, const Ctl& ctl, bool first_page_issued) {
     using L = FwdSmem<NG, S>;
-    const uint32_t kv_s = smem_addr(smem + L::kKvOff);
     const uint32_t q_s = smem_addr(smem + L::kQOff);
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
-    const uint64_t policy = p.Hg > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
+    const uint64_t policy = page_policy(p);
     WorkIter it;
     it.init(meta, p);
     Item item;
@@ -614,18 +643,10 @@ __device__ void run_producer(const CUtensorMap* kv_map, const CUtensorMap* q_map
                 continue;
             }
             MLA_TRACE_EV(kTrProdIssue);
-            int phys = __ldg(bt + j);
-            if ((unsigned)phys >= (unsigned)p.num_blocks) {
-                atomicOr(p.status, MLA_STATUS_BAD_BLOCK_TABLE);
-                phys = 0;
-            }
-            const uint32_t full = bar0 + 8 * (kKvFull0 + st);
-            mbar_arrive_expect_tx(full, L::kStageBytes);
-            const uint32_t dst = kv_s + st * L::kStageBytes;
-#pragma unroll
-            for (int c = 0; c < L::kBoxes; ++c)
-                tma_load_3d_hint(dst + c * L::kBoxBytes, kv_map, full, S::col(c, item.g, p.kv_groups), 0, phys,
-                                 policy);
+            if (first_page_issued)  // (kv_it == 0: stage 0)
+                first_page_issued = false;
+            else
+                issue_page<NG, S>(kv_map, p, item, j, st, smem, policy);
 #pragma unroll
             for (int k = 0; k < L::kStages; ++k) issued[k] += st == k;
             ++kv_it;
@@ -1262,31 +1283,32 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
 
 // The split-KV plan built inside the decode kernel from the lengths alone:
 // the same plan mla_decode_schedule_kernel writes (schedule.cuh), without its
-// launch.  The unit prefix over request-groups goes to `scratch` (BG + 1 words
-// plus 32 of warp totals, in a page stage that no copy has targeted yet);
-// this CTA's range to plan_s[0..7], with plan_s[8], plan_s[9] as the split
-// count and bad-length flag for the header.  Each CTA also writes its share of
-// the plan to the schedule buffer, for the combine kernel and for inspection:
-// its meta row; the rows of the request-groups whose first page it holds (CTA
-// 0 takes those with no pages); and CTA 0 the header and the prefix.  The
-// header's status word is left alone, so faults accumulate until the next
-// mla_decode_get_schedule clears it.  Every thread takes part; three block
-// barriers when BG fits one pass of the CTA's threads, the last one at the
-// end, after which the scratch stage is free.
-__device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, int32_t* plan_s) {
+// launch.  Two parts.  build_plan_in_cta reads only the lengths, so it runs
+// before the wait on the previous grid: the unit prefix over request-groups
+// goes to `scratch` (BG + 1 words plus 32 of warp totals, in a page stage
+// that no copy has targeted yet), this CTA's range to plan_s[0..7], and W, T
+// and the bad-length flag to plan_s[10], [11], [9].  publish_plan_in_cta runs
+// after the wait (a combine of the previous call may still read the schedule
+// buffer before it) and writes the CTA's share of the plan there, for the
+// combine kernel and for inspection: its meta row; the rows of the
+// request-groups whose first page it holds (CTA 0 takes those with no pages);
+// and CTA 0 the header and the prefix.  The header's status word is left
+// alone, so faults accumulate until the next mla_decode_get_schedule clears
+// it.  Every thread takes part in both; each ends with a block barrier (three
+// in all when BG fits one pass of the CTA's threads), the last one before the
+// scratch stage is given to the producer.
+constexpr int kPlanSlots = kMetaWords, kPlanBad = kMetaWords + 1, kPlanW = kMetaWords + 2,
+              kPlanT = kMetaWords + 3;
+
+__device__ void build_plan_in_cta(const FwdParams& p, int32_t* scratch, int32_t* plan_s) {
     const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
-    // With shared ranges every CTA of range k computes the same plan; the one
-    // of group 0 writes the range's share of it.
+    // With shared ranges every CTA of range k computes the same plan.
     const int k = blockIdx.x / p.share, G = gridDim.x / p.share, BG = p.BG, Hg = p.Hg, mb = p.max_blocks;
-    const bool writer = blockIdx.x % p.share == 0;
     int32_t* prefix = scratch;
     int32_t* warp_tot = scratch + BG + 1;
-    int32_t* meta_s = plan_s;
-    int32_t* total_slots = plan_s + kMetaWords;
-    int32_t* bad = plan_s + kMetaWords + 1;
     if (tid == 0) {
-        *total_slots = 0;
-        *bad = 0;
+        plan_s[kPlanSlots] = 0;
+        plan_s[kPlanBad] = 0;
     }
     // Unit prefix, one pass of nthr request-groups at a time: a warp scan by
     // shuffles, then every thread adds the totals of the warps before it.
@@ -1320,14 +1342,26 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
     }
     const int64_t W = carry;
     if (tid == 0) prefix[BG] = (int)W;
-    if (any_bad) *bad = 1;
+    if (any_bad) plan_s[kPlanBad] = 1;
     __syncthreads();
-    const int64_t T = units_per_cta(W, G);
     if (tid == 0) {
-        cta_meta(prefix, BG, W, T, k, meta_s);
+        const int64_t T = units_per_cta(W, G);
+        cta_meta(prefix, BG, W, T, k, plan_s);
+        plan_s[kPlanW] = (int)W;
+        plan_s[kPlanT] = (int)T;
+    }
+    __syncthreads();
+}
+
+__device__ void publish_plan_in_cta(const FwdParams& p, int NG, const int32_t* scratch, int32_t* plan_s) {
+    const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31;
+    const int k = blockIdx.x / p.share, G = gridDim.x / p.share, BG = p.BG, Hg = p.Hg;
+    const bool writer = blockIdx.x % p.share == 0;  // group 0 of a shared range writes its rows
+    const int32_t* prefix = scratch;
+    const int64_t T = plan_s[kPlanT];
+    if (tid == 0 && writer) {
         int32_t* row = p.plan_out + kHdrWords + (size_t)k * kMetaWords;
-        if (writer)
-            for (int i = 0; i < kMetaWords; ++i) row[i] = meta_s[i];
+        for (int i = 0; i < kMetaWords; ++i) row[i] = plan_s[i];
     }
     int32_t* bginfo = p.plan_out + bg_offset_words(G);
     int my_slots = 0;
@@ -1347,7 +1381,7 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
         for (int i = tid; i <= BG; i += nthr) pg[i] = prefix[i];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) my_slots += __shfl_xor_sync(kFullMask, my_slots, o);
-        if (lane == 0 && my_slots) atomicAdd(total_slots, my_slots);
+        if (lane == 0 && my_slots) atomicAdd(plan_s + kPlanSlots, my_slots);
     }
     __syncthreads();
     if (blockIdx.x == 0 && tid == 0) {
@@ -1357,15 +1391,15 @@ __device__ void build_plan_in_cta(const FwdParams& p, int NG, int32_t* scratch, 
         h[kHdrBG] = BG;
         h[kHdrHg] = Hg;
         h[kHdrNG] = NG;
-        h[kHdrSlots] = *total_slots;
+        h[kHdrSlots] = plan_s[kPlanSlots];
         h[kHdrT] = (int)T;
-        h[kHdrW] = (int)W;
+        h[kHdrW] = plan_s[kPlanW];
         h[kHdrBatch] = BG / Hg;
-        h[kHdrMaxBlocks] = mb;
+        h[kHdrMaxBlocks] = p.max_blocks;
         h[kHdrShift] = kPageShift;
         h[kHdrShareHg] = p.share;
         for (int i = kHdrShareHg + 1; i < kHdrWords; ++i) h[i] = 0;
-        if (*bad) atomicOr(p.status, MLA_STATUS_BAD_SEQLEN);
+        if (plan_s[kPlanBad]) atomicOr(p.status, MLA_STATUS_BAD_SEQLEN);
     }
 }
 
@@ -1381,6 +1415,9 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     MLA_TRACE_K(0);
+    // The grid after this one (the combine) may launch now: it waits for this
+    // grid's end before it reads anything of it.
+    griddep_launch_dependents();
     const uint32_t bar0 = smem_addr(smem + L::kBarOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -1420,11 +1457,35 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // A plan built here is computed from the lengths alone before the wait
+    // below, while the grid before this one (for example the query
+    // projection) finishes; the second page stage holds its scratch until the
+    // producer's first copy into it, after publish_plan_in_cta.  The lengths
+    // must be final when that grid lets its dependents start.
+    int32_t* plan_scratch = reinterpret_cast<int32_t*>(smem + L::kKvOff + L::kStageBytes);
+    bool first_page_issued = false;
+    if (p.plan_out != nullptr && !misaligned) {
+        build_plan_in_cta(p, plan_scratch, meta_s);
+        // With the range known, the producer thread starts the first page of
+        // its first item into stage 0 before the wait as well: the cache and
+        // the block table, like the lengths, must be final when the grid
+        // before this one lets its dependents start.
+        if (threadIdx.x == 0 && p.test_stall == 0) {
+            WorkIter it;
+            it.init(meta_s, p);
+            Item item;
+            // (a bad block-table entry is left to the producer, which reports
+            // it after the wait: the status word may still be reset before it)
+            if (it.next(p, item) &&
+                (unsigned)__ldg(p.block_table + (size_t)item.b * p.max_blocks + item.p0) < (unsigned)p.num_blocks) {
+                issue_page<NG, S>(&kv_map, p, item, item.p0, 0, smem, page_policy(p));
+                first_page_issued = true;
+            }
+        }
+    }
     // Launched as a programmatic dependent: wait until the grid before this
-    // one (the schedule kernel, or whatever wrote q and the lengths) is
-    // complete, then let the combine launch behind this grid.
+    // one (the schedule kernel, or whatever wrote q) is complete.
     griddep_wait();
-    griddep_launch_dependents();
     MLA_TRACE_K(1);
     if (misaligned) {
         if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_SMEM_ALIGN);
@@ -1433,16 +1494,13 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int32_t* meta;
     if (p.plan_out != nullptr) {
-        // The plan is built here; the second page stage holds its scratch
-        // until the producer's first copy into it, after the barrier that
-        // ends build_plan_in_cta.
-        build_plan_in_cta(p, NG, reinterpret_cast<int32_t*>(smem + L::kKvOff + L::kStageBytes), meta_s);
+        publish_plan_in_cta(p, NG, plan_scratch, meta_s);
         meta = meta_s;
     } else {
         const int32_t* hdr = p.sched;
-        if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
-            __ldg(hdr + kHdrBG) != p.BG || __ldg(hdr + kHdrHg) != p.Hg || __ldg(hdr + kHdrNG) != NG ||
-            __ldg(hdr + kHdrShift) != kPageShift || __ldg(hdr + kHdrShareHg) != p.share) {
+        if (hdr[kHdrMagic] != kSchedMagic || hdr[kHdrG] != p.G ||
+            hdr[kHdrBG] != p.BG || hdr[kHdrHg] != p.Hg || hdr[kHdrNG] != NG ||
+            hdr[kHdrShift] != kPageShift || hdr[kHdrShareHg] != p.share) {
             if (threadIdx.x == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
             if (warp == 1) {
                 tc_fence_after();
@@ -1461,7 +1519,7 @@ __global__ void __launch_bounds__(FwdWarps<NG, S>::kThreads, 1)
             if (lane == 0) {
                 prefetch_tensormap(&kv_map);
                 prefetch_tensormap(&q_map);
-                run_producer<NG, S>(&kv_map, &q_map, p, meta, smem, ctl);
+                run_producer<NG, S>(&kv_map, &q_map, p, meta, smem, ctl, first_page_issued);
             }
         } else if (warp <= G1<NG>::kIssuers) {
             if (lane == 0) run_gemm1<NG, S>(p, meta, smem, tmem, ctl, warp - 1);
@@ -1529,14 +1587,21 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     __shared__ float wts[kCombineThreads];
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
+    // The grid after this one (the output projection, or the next decode) may
+    // start its prologue now; it reads nothing of this grid's before its own
+    // wait for this grid's completion.
+    griddep_launch_dependents();
     // A plan from the schedule kernel may be read before the wait: the decode
     // grid let this grid start only after its own wait on the grid that wrote
     // it.  A plan the decode kernel built itself is complete only after it.
+    // What an earlier grid wrote (the plan, the partials) is read with plain
+    // loads: a read-only __ldg load may be scheduled above the wait, and one
+    // was (a combine that read the header before the decode grid wrote it).
     if (p.plan_in_decode) griddep_wait();
     const int32_t* hdr = p.sched;
-    if (__ldg(hdr + kHdrMagic) != kSchedMagic || __ldg(hdr + kHdrG) != p.G ||
-        __ldg(hdr + kHdrBG) != p.plan_BG || __ldg(hdr + kHdrHg) != p.plan_Hg || __ldg(hdr + kHdrNG) != p.NG ||
-        __ldg(hdr + kHdrShift) != p.shift || __ldg(hdr + kHdrShareHg) != p.share) {
+    if (hdr[kHdrMagic] != kSchedMagic || hdr[kHdrG] != p.G ||
+        hdr[kHdrBG] != p.plan_BG || hdr[kHdrHg] != p.plan_Hg || hdr[kHdrNG] != p.NG ||
+        hdr[kHdrShift] != p.shift || hdr[kHdrShareHg] != p.share) {
         if (threadIdx.x == 0 && bg == 0 && n == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }
@@ -1548,8 +1613,8 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     const int row = p.share > 1 ? b : bg;  // plan row of this request-group
     const int gs = p.share > 1 ? g : 0;
     const int32_t* info = hdr + bg_offset_words(p.G) + (size_t)kBgWords * row;
-    const int base = __ldg(info + 0);
-    const int k = __ldg(info + 1);
+    const int base = info[0];
+    const int k = info[1];
     if (k == 1) return;  // unsplit: the decode kernel wrote the final row
     // Slots of the splits: the one-CTA kernels' fixed slots (split_slot, times
     // the groups sharing a range, plus the group), or the CTA-pair plans'
@@ -1570,8 +1635,8 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     auto slot_i = [&](int i) -> size_t { return i == 0 ? slot0 : slot1 + (size_t)(i - 1) * sstride; };
     const float* lp0 = p.lpart + n;
     const float* op0 = p.opart + (size_t)n * kDv + d0;
-    auto lse_of = [&](int i) { return __ldg(lp0 + slot_i(i) * p.NG); };
-    auto row_of = [&](int i) { return __ldg(reinterpret_cast<const float4*>(op0 + slot_i(i) * p.NG * kDv)); };
+    auto lse_of = [&](int i) { return lp0[slot_i(i) * p.NG]; };
+    auto row_of = [&](int i) { return *reinterpret_cast<const float4*>(op0 + slot_i(i) * p.NG * kDv); };
     MLA_TRACE_STEP_MIN(2);
     if (!p.plan_in_decode) griddep_wait();  // the decode grid's partials are complete and visible
     MLA_TRACE_STEP_MIN(3);
