@@ -130,11 +130,11 @@ struct PairIter {
     int b, begin_b, begin_s, end_b, end_s, first_split;
 
     __device__ void init(const int32_t* meta) {
-        begin_b = meta[kMetaBeginBg];
-        begin_s = meta[kMetaBeginPage];
-        end_b = meta[kMetaEndBg];
-        end_s = meta[kMetaEndPage];
-        first_split = meta[kMetaFirstSplit];
+        begin_b = ld_nc_after_wait(meta + kMetaBeginBg);
+        begin_s = ld_nc_after_wait(meta + kMetaBeginPage);
+        end_b = ld_nc_after_wait(meta + kMetaEndBg);
+        end_s = ld_nc_after_wait(meta + kMetaEndPage);
+        first_split = ld_nc_after_wait(meta + kMetaFirstSplit);
         b = begin_b;
     }
 
@@ -157,7 +157,7 @@ struct PairIter {
             it.unsplit = (s0 == 0 && s1 == S);
             it.slot = -1;
             if (!it.unsplit) {
-                const int s = bginfo[kBgWords * cur] + ((cur == begin_b) ? first_split : 0);
+                const int s = ld_nc_after_wait(bginfo + kBgWords * cur) + ((cur == begin_b) ? first_split : 0);
                 const int slot = s * p.Hg + g;
                 it.slot = (s >= 0 && slot < p.slots_cap) ? slot : -1;
             }
@@ -633,9 +633,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // Both CTAs of the cluster read the same header and take the same exits.
     const int32_t* hdr = p.sched;
     const int cluster = blockIdx.x >> 1;
-    if (hdr[kHdrMagic] != kSchedMagic || hdr[kHdrG] != p.G || hdr[kHdrBG] != p.BG ||
-        hdr[kHdrHg] != 1 || hdr[kHdrNG] != kPairCols || hdr[kHdrShift] != kStepShift ||
-        hdr[kHdrShareHg] != p.Hg) {
+    auto h = [&](int i) { return ld_nc_after_wait(hdr + i); };
+    if (h(kHdrMagic) != kSchedMagic || h(kHdrG) != p.G || h(kHdrBG) != p.BG || h(kHdrHg) != 1 ||
+        h(kHdrNG) != kPairCols || h(kHdrShift) != kStepShift || h(kHdrShareHg) != p.Hg) {
         if (threadIdx.x == 0 && rank == 0) atomicOr(p.status, MLA_STATUS_BAD_SCHEDULE);
         return;
     }

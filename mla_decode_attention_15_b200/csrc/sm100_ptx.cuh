@@ -30,6 +30,16 @@ __device__ __forceinline__ uint64_t stamp_timer_ns() {
     return t;
 }
 
+// Read-only load of a word an earlier grid wrote, for use after the
+// grid-dependency wait: the read-only path like __ldg, but as a volatile asm
+// statement the compiler keeps after the (volatile) wait, where an __ldg may be
+// scheduled above it.
+__device__ __forceinline__ int32_t ld_nc_after_wait(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // Prefetch of one global line into L2 (no data returned; safe while another
 // grid may still write the line, since the later real load reads L2).
 __device__ __forceinline__ void prefetch_l2_line(const void* gptr) {

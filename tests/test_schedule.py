@@ -120,10 +120,11 @@ def test_plan_long_single_request_spreads_over_all_ctas():
 
 
 def test_plan_short_batch_uses_few_ctas():
-    pl = host_plan([1024], 1, 16, 148)  # 16 pages
+    pl = host_plan([1024], 1, 16, 148)  # 16 pages: 17 units, at least 2 per range (1 page + the item's unit)
     items = check_invariants(pl)
     busy = [its for its in items if its]
-    assert 2 <= len(busy) <= 8
+    assert int(pl["hdr"][6]) == 2
+    assert len(busy) == 9
     assert all(p1 - p0 >= 1 for its in busy for (_, p0, p1, _, _) in its)
 
 
