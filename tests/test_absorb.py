@@ -133,8 +133,9 @@ def test_absorb_wrappers_and_streams(dev):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("inline", [False, True])
 @pytest.mark.parametrize("heads,s_q,causal", [(16, 1, False), (128, 2, True)])
-def test_absorbed_decode_step_matches_oracle_chain(dev, heads, s_q, causal):
+def test_absorbed_decode_step_matches_oracle_chain(dev, heads, s_q, causal, inline):
     """absorb_q -> decode over the latent cache -> absorb_o through the C
     ABI, step by step, against the oracle chain started from the GPU's own
     latent query (whose projection is checked element by element in the
@@ -144,7 +145,10 @@ def test_absorbed_decode_step_matches_oracle_chain(dev, heads, s_q, causal):
       - each element of the projected output is within the error the decode
         carried into it, pushed through W_UV exactly (|e| . |W_UV|), plus one
         bf16 rounding of the result and the fp32 summation of 512 products;
-      - the one-call chain ``absorbed_mla_decode`` gives the same bits."""
+      - the one-call chain ``absorbed_mla_decode`` gives the same bits.
+    With ``inline`` the decode builds its plan and loads its first pages
+    while the query projection before it (which lets its dependents start
+    early) is still running: it must still read the projected query."""
     import oracle
     from oracle import absorb
     lens = [1, 70, 1000, 2500]
@@ -155,7 +159,8 @@ def test_absorbed_decode_step_matches_oracle_chain(dev, heads, s_q, causal):
     q_in = x["q_in"].view(B, s_q, heads, 192)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
     w_uk, w_uv = x["w_uk"].to(dev), x["w_uv"].to(dev)
-    dec = bd.MlaDecoder(B, s_q, heads, g["kv_cache"].shape[0], g["block_table"].shape[1], causal, 0, dev)
+    dec = bd.MlaDecoder(B, s_q, heads, g["kv_cache"].shape[0], g["block_table"].shape[1], causal, 0, dev,
+                        inline_plan=inline)
     dec.plan(g["cache_seqlens"])
     q_lat = bd.absorb_q(q_in.to(dev), w_uk)
     o_lat, lse = dec(q_lat, g["kv_cache"], g["block_table"], g["cache_seqlens"], d["softmax_scale"])
