@@ -1553,8 +1553,9 @@ constexpr int kCombinePre = 8;
 constexpr int kCombineUnroll = 8;
 // Up to this many splits the merge takes no block reduction.  Measured on
 // B200 (graph-replayed steps): at 4 the 128-head workload's ~8,200 combine
-// CTAs (2-3 splits each) take 8 us less than with block reductions, while
-// raising it to 8 costs the ragged 16-head workload ~4 us.
+// CTAs (2-3 splits each) take 8 us less than with block reductions; at 8 the
+// larger arrays cost registers, fewer combine CTAs share an SM, and that
+// step is 4 us slower than at 4 (the 16-head workloads were unchanged).
 constexpr int kCombineFast = 4;
 
 template <int kCombineThreads, bool kMax>
