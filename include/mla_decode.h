@@ -253,6 +253,11 @@ size_t mla_gqa_decode_schedule_bytes(const mla_gqa_dims* dims);
 size_t mla_gqa_decode_workspace_bytes(const mla_gqa_dims* dims);
 int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_seqlens, void* schedule,
                                 void* stream);
+/* The same GQA plan computed on the host from host arrays (for inspection and
+ * tests); `schedule_host` is host memory of mla_gqa_decode_schedule_bytes(dims)
+ * bytes.  dims->num_sms must be > 0.  No CUDA call is made. */
+int mla_gqa_decode_get_schedule_host(const mla_gqa_dims* dims, const int32_t* cache_seqlens_host,
+                                     void* schedule_host);
 int mla_gqa_decode_fwd(const mla_gqa_dims* dims, void* schedule, void* workspace, const void* q,
                        const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
                        float softmax_scale, void* out, float* lse, void* stream);

@@ -37,6 +37,7 @@ from .binding import (  # noqa: F401
     mla_gqa_decode_combine,
     mla_gqa_decode_fwd,
     mla_gqa_decode_get_schedule,
+    mla_gqa_decode_get_schedule_host,
     mla_gqa_decode_schedule_bytes,
     mla_gqa_decode_workspace_bytes,
 )

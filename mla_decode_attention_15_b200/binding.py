@@ -52,6 +52,7 @@ EXPORTED = (
     "mla_gqa_decode_schedule_bytes",
     "mla_gqa_decode_workspace_bytes",
     "mla_gqa_decode_get_schedule",
+    "mla_gqa_decode_get_schedule_host",
     "mla_gqa_decode_fwd",
     "mla_gqa_decode_combine",
     "mla_absorb_q",
@@ -137,6 +138,8 @@ def lib() -> ctypes.CDLL:
         L.mla_gqa_decode_workspace_bytes.argtypes = [Q]
         L.mla_gqa_decode_get_schedule.restype = ctypes.c_int
         L.mla_gqa_decode_get_schedule.argtypes = [Q, vp, vp, vp]
+        L.mla_gqa_decode_get_schedule_host.restype = ctypes.c_int
+        L.mla_gqa_decode_get_schedule_host.argtypes = [Q, vp, vp]
         L.mla_gqa_decode_fwd.restype = ctypes.c_int
         L.mla_gqa_decode_fwd.argtypes = [Q, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
         L.mla_gqa_decode_combine.restype = ctypes.c_int
@@ -331,6 +334,12 @@ def mla_gqa_decode_workspace_bytes(dims: mla_gqa_dims) -> int:
 def mla_gqa_decode_get_schedule(dims, cache_seqlens, schedule, stream=None) -> None:
     _check(lib().mla_gqa_decode_get_schedule(ctypes.byref(dims), _ptr(cache_seqlens), _ptr(schedule),
                                              _stream(stream)), "mla_gqa_decode_get_schedule")
+
+
+def mla_gqa_decode_get_schedule_host(dims, cache_seqlens, schedule) -> None:
+    """Host version; ``cache_seqlens`` (int32) and ``schedule`` are CPU tensors."""
+    _check(lib().mla_gqa_decode_get_schedule_host(ctypes.byref(dims), _ptr(cache_seqlens), _ptr(schedule)),
+           "mla_gqa_decode_get_schedule_host")
 
 
 def mla_gqa_decode_fwd(dims, schedule, workspace, q, kv_cache, block_table, cache_seqlens,

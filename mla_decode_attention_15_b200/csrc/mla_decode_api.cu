@@ -516,6 +516,47 @@ int launch_absorb(const mla_absorb_dims* d, const void* x, const void* w, void* 
 
 }  // namespace
 
+// The split-KV plan computed on the host, word for word what the schedule
+// kernel writes (schedule.cuh); for inspection and tests.
+void host_plan(const Plan& pl, int batch, int mb, const int32_t* seqlens, void* schedule_host) {
+    const int G = pl.G, BG = pl.BG, Hg = pl.plan_Hg, sh = pl.shift;
+    int32_t* s = static_cast<int32_t*>(schedule_host);
+    int32_t* prefix = s + prefix_offset_words(G, BG);
+    int32_t* bginfo = s + bg_offset_words(G);
+    int bad_len = 0;
+    int64_t W = 0;
+    for (int bg = 0; bg < BG; ++bg) {
+        const int L = seqlens[bg / Hg];
+        if (!seqlen_in_range(L, mb)) bad_len = 1;
+        prefix[bg] = (int32_t)W;
+        W += units_of(blocks_of(clamp_seqlen(L, mb), sh));
+    }
+    prefix[BG] = (int32_t)W;
+    const int64_t T = units_per_cta(W, G);
+    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, s + kHdrWords + (size_t)k * kMetaWords);
+    int64_t slots = 0;
+    for (int bg = 0; bg < BG; ++bg) {
+        const int ns = num_splits_of(prefix, bg, pages_in_prefix(prefix, bg), T);
+        bginfo[kBgWords * bg] = pl.pair ? (int32_t)slots : ns > 1 ? first_split_slot(prefix, bg, T) : 0;
+        bginfo[kBgWords * bg + 1] = ns;
+        if (ns > 1) slots += ns;
+    }
+    std::memset(s, 0, kHdrWords * sizeof(int32_t));
+    s[kHdrMagic] = kSchedMagic;
+    s[kHdrG] = G;
+    s[kHdrBG] = BG;
+    s[kHdrHg] = Hg;
+    s[kHdrNG] = pl.gr.NG;
+    s[kHdrSlots] = (int32_t)slots;
+    s[kHdrT] = (int32_t)T;
+    s[kHdrStatus] = bad_len ? MLA_STATUS_BAD_SEQLEN : 0;
+    s[kHdrW] = (int32_t)W;
+    s[kHdrBatch] = batch;
+    s[kHdrMaxBlocks] = mb;
+    s[kHdrShift] = sh;
+    s[kHdrShareHg] = pl.share;
+}
+
 extern "C" {
 
 int mla_decode_version(void) { return kAbiVersion; }
@@ -564,43 +605,7 @@ int mla_decode_get_schedule_host(const mla_decode_dims* dims, const int32_t* seq
     Plan pl;
     rc = make_plan(dims, &pl);
     if (rc != MLA_OK) return rc;
-    const Grouping gr = pl.gr;
-    const int G = pl.G, BG = pl.BG, Hg = pl.plan_Hg, sh = pl.shift, mb = dims->max_blocks_per_seq;
-    int32_t* s = static_cast<int32_t*>(schedule_host);
-    int32_t* prefix = s + prefix_offset_words(G, BG);
-    int32_t* bginfo = s + bg_offset_words(G);
-    int bad_len = 0;
-    int64_t W = 0;
-    for (int bg = 0; bg < BG; ++bg) {
-        const int L = seqlens[bg / Hg];
-        if (!seqlen_in_range(L, mb)) bad_len = 1;
-        prefix[bg] = (int32_t)W;
-        W += units_of(blocks_of(clamp_seqlen(L, mb), sh));
-    }
-    prefix[BG] = (int32_t)W;
-    const int64_t T = units_per_cta(W, G);
-    for (int k = 0; k < G; ++k) cta_meta(prefix, BG, W, T, k, s + kHdrWords + (size_t)k * kMetaWords);
-    int64_t slots = 0;
-    for (int bg = 0; bg < BG; ++bg) {
-        const int ns = num_splits_of(prefix, bg, pages_in_prefix(prefix, bg), T);
-        bginfo[kBgWords * bg] = pl.pair ? (int32_t)slots : ns > 1 ? first_split_slot(prefix, bg, T) : 0;
-        bginfo[kBgWords * bg + 1] = ns;
-        if (ns > 1) slots += ns;
-    }
-    std::memset(s, 0, kHdrWords * sizeof(int32_t));
-    s[kHdrMagic] = kSchedMagic;
-    s[kHdrG] = G;
-    s[kHdrBG] = BG;
-    s[kHdrHg] = Hg;
-    s[kHdrNG] = gr.NG;
-    s[kHdrSlots] = (int32_t)slots;
-    s[kHdrT] = (int32_t)T;
-    s[kHdrStatus] = bad_len ? MLA_STATUS_BAD_SEQLEN : 0;
-    s[kHdrW] = (int32_t)W;
-    s[kHdrBatch] = dims->batch;
-    s[kHdrMaxBlocks] = mb;
-    s[kHdrShift] = sh;
-    s[kHdrShareHg] = pl.share;
+    host_plan(pl, dims->batch, dims->max_blocks_per_seq, seqlens, schedule_host);
     return MLA_OK;
 }
 
@@ -694,6 +699,17 @@ int mla_gqa_decode_get_schedule(const mla_gqa_dims* dims, const int32_t* cache_s
     if (!aligned16(cache_seqlens) || !aligned16(schedule)) return MLA_ERR_INVALID_ARG;
     return launch_schedule(pl, dims->batch, dims->max_blocks_per_seq, cache_seqlens, schedule,
                            static_cast<cudaStream_t>(stream));
+}
+
+int mla_gqa_decode_get_schedule_host(const mla_gqa_dims* dims, const int32_t* seqlens, void* schedule_host) {
+    int rc = validate_gqa(dims);
+    if (rc != MLA_OK) return rc;
+    if (dims->num_sms <= 0 || seqlens == nullptr || schedule_host == nullptr) return MLA_ERR_INVALID_ARG;
+    Plan pl;
+    rc = make_plan_gqa(dims, &pl);
+    if (rc != MLA_OK) return rc;
+    host_plan(pl, dims->batch, dims->max_blocks_per_seq, seqlens, schedule_host);
+    return MLA_OK;
 }
 
 int mla_gqa_decode_fwd(const mla_gqa_dims* dims, void* schedule, void* workspace, const void* q,

@@ -213,3 +213,28 @@ def test_poisoned_workspace_and_outputs(dev):
     ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
                                    d["softmax_scale"], causal=True)
     helpers.compare(out, lse, ro, rl)
+
+
+@pytest.mark.parametrize("groups,G", [(8, 148), (2, 148), (8, 7), (1, 148)])
+def test_gqa_written_plan_equals_host_plan(dev, groups, G):
+    """The GQA plan built in the decode kernel (shared ranges for 2 and 8 KV
+    groups on 148 SMs; one row per request-group for 8 groups on 7 SMs and
+    for one group) equals the host plan word for word."""
+    lens = [0, 5, 64, 65, 9000, 1, 130, 2500]
+    d = workloads.build_gqa(len(lens), 2, groups, ("list", lens), seed=31 + groups, causal=True)
+    g = to_dev(d, dev)
+    dec = bd.GqaDecoder(len(lens), 2, groups, g["kv_cache"].shape[0], g["block_table"].shape[1], True, G, dev,
+                        inline_plan=True)
+    dec.plan(g["cache_seqlens"])
+    words = dec.schedule.view(torch.int32)
+    words[:HDR_STATUS] = 0x7FAB7FAB
+    words[HDR_STATUS + 1:] = 0x7FAB7FAB
+    dec(g["q"], g["kv_cache"], g["block_table"], g["cache_seqlens"], g["softmax_scale"])
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    host = torch.zeros(dec.schedule.numel(), dtype=torch.uint8)
+    bd.mla_gqa_decode_get_schedule_host(dec.dims, d["cache_seqlens"], host)
+    got = dec.schedule.cpu().view(torch.int32).numpy()
+    want = host.view(torch.int32).numpy()
+    diff = np.nonzero(got != want)[0]
+    assert diff.size == 0, (diff[:10], got[diff[:10]], want[diff[:10]])

@@ -137,3 +137,41 @@ def test_plan_clamps_and_flags_bad_lengths():
     assert total == 4                            # clamped to the table's 4 pages
     ok = host_plan([100, 5], 1, 16, 8, max_blocks=4)
     assert ok["hdr"][7] == 0
+
+
+def gqa_host_plan(seqlens, s_q, groups, G, max_blocks=None):
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int32).contiguous()
+    B = seqlens.numel()
+    if max_blocks is None:
+        max_blocks = max(1, (int(seqlens.clamp(min=0).max()) + 63) // 64)
+    d = bd.make_gqa_dims(B, s_q, groups, 10 ** 6, max_blocks, s_q > 1, G)
+    buf = torch.zeros(bd.mla_gqa_decode_schedule_bytes(d), dtype=torch.uint8)
+    bd.mla_gqa_decode_get_schedule_host(d, seqlens, buf)
+    if groups > 1 and G // groups >= 1:   # shared ranges: one plan row per request
+        Gp, BG, Hg, share = G // groups, B, 1, groups
+    else:                                 # one plan row per request-group
+        Gp, BG, Hg, share = G, B * groups, groups, 1
+    words = buf.numpy().view(np.int32)
+    assert (int(words[1]), int(words[2]), int(words[3]), int(words[4]), int(words[11]), int(words[12])) == \
+        (Gp, BG, Hg, 16 * s_q, 6, share)
+    hdr, meta, bginfo, prefix = helpers.read_plan(buf.numpy(), Gp, BG)
+    return dict(hdr=hdr, meta=meta, bginfo=bginfo, prefix=prefix, Hg=Hg, BG=BG, G=Gp, shift=6, share=share,
+                seqlens=seqlens.numpy(), max_blocks=max_blocks)
+
+
+@pytest.mark.parametrize("G", [1, 7, 16, 148])
+@pytest.mark.parametrize("groups", [1, 2, 8])
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_gqa_plan_random_ragged(G, groups, s_q):
+    """The GQA plan: with several KV groups (and at least one range per group)
+    one row per request, each range walked by all groups; every page of every
+    request once, partial slots unique and split counts consistent."""
+    rng = np.random.default_rng(G * 100 + groups * 10 + s_q)
+    lens = rng.integers(0, 5000, size=int(rng.integers(1, 30))).tolist()
+    lens[0] = 0
+    pl = gqa_host_plan(lens, s_q, groups, G)
+    check_invariants(pl)
+    # the slots a shared range's CTAs write (fixed slot x groups + group) fit the workspace
+    d = bd.make_gqa_dims(len(lens), s_q, groups, 10 ** 6, pl["max_blocks"], s_q > 1, G)
+    slot_bytes = 16 * s_q * (128 + 1) * 4
+    assert bd.mla_gqa_decode_workspace_bytes(d) == 2 * pl["G"] * pl["share"] * slot_bytes
