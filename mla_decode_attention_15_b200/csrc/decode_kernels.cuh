@@ -1557,6 +1557,20 @@ constexpr int kCombineUnroll = 8;
 // larger arrays cost registers, fewer combine CTAs share an SM, and that
 // step is 4 us slower than at 4 (the 16-head workloads were unchanged).
 constexpr int kCombineFast = 4;
+// Many splits with few combine CTAs (a short batch over a long context: one
+// request over 148 CTAs has ~148 splits in 16 CTAs) make the per-thread chain
+// of row loads the step's tail: measured on B200 (graph-replayed, L2 flushed),
+// a bs1 x 16K step took 46.5 us against 18.5 us for its decode alone.  When
+// the combine grid (one CTA per request-group and column) is smaller than the
+// decode grid, the host launches kCombineSlices CTAs per column (grid z).
+// Above kCombineSliceMin splits, CTA z then merges d_v columns
+// [z * 128, z * 128 + 128) only: lane l owns four of them, and warp w takes
+// splits w, w + 4, ..., kCombineUnroll rows in flight.  Each thread walks a
+// quarter of the splits, on four times as many SMs.  The four warps' sums
+// meet in shared memory, in warp order.  Up to kCombineSliceMin splits, CTA 0
+// merges the whole row as above and the others leave.
+constexpr int kCombineSlices = 4;
+constexpr int kCombineSliceMin = 16;
 
 template <int kCombineThreads, bool kMax>
 __device__ __forceinline__ float combine_block_reduce(float v, float* red) {
@@ -1581,11 +1595,15 @@ __device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
     acc.w = fmaf(w, v.w, acc.w);
 }
 
-template <int kDv>
+template <int kDv, bool kSliced>
 __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const CombineParams p) {
     constexpr int kCombineThreads = kDv / 4;
-    __shared__ float red[kCombineThreads / 32];
+    constexpr int kWarps = kCombineThreads / 32;
+    // the sliced launch only; a warp's lanes cover one slice
+    constexpr bool kCanSlice = kSliced && kDv == kCombineSlices * 32 * 4;
+    __shared__ float red[kWarps];
     __shared__ float wts[kCombineThreads];
+    __shared__ float4 wsum[kWarps][32];
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
     // The grid after this one (the output projection, or the next decode) may
@@ -1617,6 +1635,8 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
     const int base = info[0];
     const int k = info[1];
     if (k == 1) return;  // unsplit: the decode kernel wrote the final row
+    const bool sliced = kCanSlice && gridDim.z > 1 && k > kCombineSliceMin;
+    if (!sliced && blockIdx.z != 0) return;  // CTA 0 of the column merges the whole row
     // Slots of the splits: the one-CTA kernels' fixed slots (split_slot, times
     // the groups sharing a range, plus the group), or the CTA-pair plans'
     // (base + i) * share + group.  In both, split i >= 1 sits at a constant
@@ -1669,6 +1689,49 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
             for (int i = 0; i < kCombineFast; ++i)
                 if (i < k) fma4(acc, expf(l[i] - lstar), v[i]);
         }
+    } else if (sliced) {
+        float own = threadIdx.x < k ? lse_of(threadIdx.x) : -INFINITY;
+        float mx = own;
+        for (int i = threadIdx.x + kCombineThreads; i < k; i += kCombineThreads) mx = fmaxf(mx, lse_of(i));
+        mx = combine_block_reduce<kCombineThreads, true>(mx, red);
+        if (mx != -INFINITY) {  // uniform across the block
+            float sum = 0.f;
+            for (int i = threadIdx.x; i < k; i += kCombineThreads)
+                sum += expf((i == threadIdx.x ? own : lse_of(i)) - mx);
+            sum = combine_block_reduce<kCombineThreads, false>(sum, red);
+            lstar = mx + logf(sum);
+            const int warp = threadIdx.x >> 5;
+            const float* rs = p.opart + (size_t)n * kDv + blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x & 31) * 4;
+            auto srow = [&](int i) { return *reinterpret_cast<const float4*>(rs + slot_i(i) * p.NG * kDv); };
+            for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
+                const int cn = k - c0 < kCombineThreads ? k - c0 : kCombineThreads;
+                __syncthreads();  // the previous chunk's weights are consumed
+                if (threadIdx.x < cn) wts[threadIdx.x] = expf((c0 == 0 ? own : lse_of(c0 + threadIdx.x)) - lstar);
+                __syncthreads();
+                int j = warp;
+                for (; j + kWarps * (kCombineUnroll - 1) < cn; j += kWarps * kCombineUnroll) {
+                    float4 v[kCombineUnroll];
+#pragma unroll
+                    for (int u = 0; u < kCombineUnroll; ++u) v[u] = srow(c0 + j + kWarps * u);
+#pragma unroll
+                    for (int u = 0; u < kCombineUnroll; ++u) fma4(acc, wts[j + kWarps * u], v[u]);
+                }
+                for (; j < cn; j += kWarps) fma4(acc, wts[j], srow(c0 + j));
+            }
+        }
+        wsum[threadIdx.x >> 5][threadIdx.x & 31] = acc;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            acc = wsum[0][threadIdx.x];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {
+                const float4 t = wsum[w][threadIdx.x];
+                acc.x += t.x;
+                acc.y += t.y;
+                acc.z += t.z;
+                acc.w += t.w;
+            }
+        }
     } else if (k > 1) {
         float4 pre[kCombinePre];
 #pragma unroll
@@ -1707,18 +1770,21 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
             }
         }
     }
-    const size_t o = (((size_t)b * p.s_q + s) * p.heads + head) * kDv + d0;
-    if (p.out_f32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = acc;
-    } else {
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 packed;
-        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) = packed;
+    const int dcol = sliced ? (int)blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x & 31) * 4 : d0;
+    const size_t o = (((size_t)b * p.s_q + s) * p.heads + head) * kDv + dcol;
+    if (!sliced || threadIdx.x < 32) {
+        if (p.out_f32) {
+            *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = acc;
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 packed;
+            packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+            packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) = packed;
+        }
     }
-    if (threadIdx.x == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
+    if (threadIdx.x == 0 && blockIdx.z == 0) p.lse[((size_t)b * p.heads + head) * p.s_q + s] = lstar;
     MLA_TRACE_STEP_MAX(4);
 #ifdef MLA_TRACE
     if (threadIdx.x == 0 && bg < 64 && n < 64) g_mla_trace_comb[bg][n] = stamp_timer_ns();

@@ -354,7 +354,10 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
     c.run_rows = cm.run_rows;
     c.run_stride = cm.run_stride;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(c.BG, pl.gr.NG);
+    // Fewer combine CTAs than decode CTAs: several per column, so that many
+    // splits are merged in d_v slices (mla_decode_combine_kernel).
+    const bool slices = kDvT == kCombineSlices * 128 && (int64_t)c.BG * pl.gr.NG < pl.ctas;
+    cfg.gridDim = dim3(c.BG, pl.gr.NG, slices ? kCombineSlices : 1);
     cfg.blockDim = dim3(kDvT / 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -363,7 +366,9 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel<kDvT>, c) != cudaSuccess) {
+    const cudaError_t e = slices ? cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel<kDvT, true>, c)
+                                 : cudaLaunchKernelEx(&cfg, mla_decode_combine_kernel<kDvT, false>, c);
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }

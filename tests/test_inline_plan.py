@@ -76,6 +76,17 @@ def test_ragged_heads_and_grids_match_two_launch_path(dev, heads, s_q, num_sms):
     same_as_two_launch_path(d, dev, num_sms)
 
 
+@pytest.mark.parametrize("lens,s_q", [([66000], 1), ([9000, 3000], 2)])
+def test_many_splits_match_two_launch_path_and_oracle(dev, lens, s_q):
+    """Short batches over long contexts: 148, 71 and 24 splits per column,
+    merged in d_v slices by the small combine grid."""
+    d = workloads.build(len(lens), s_q, 16, ("list", lens), seed=9 + s_q, causal=s_q > 1)
+    out, lse = same_as_two_launch_path(d, dev, 148)
+    ro, rl = oracle.mla_oracle_fwd(d["q"], d["kv_cache"], d["block_table"], d["cache_seqlens"],
+                                   d["softmax_scale"], causal=d["causal"])
+    helpers.compare(out, lse, ro, rl)
+
+
 def test_fp32_output_matches_two_launch_path(dev):
     lens = [5000, 64, 2222, 1]
     d = workloads.build(len(lens), 2, 16, ("list", lens), seed=17, causal=True)

@@ -272,6 +272,47 @@ def test_explicit_combine_matches_fused_launch(dev):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# Short batches over long contexts: many splits per column in a small combine
+# grid, which the library merges in d_v slices (four CTAs per column).  The
+# split counts in the comments are the plan's at 148 CTAs.
+@pytest.mark.parametrize("lens,s_q,heads", [
+    ([66000], 1, 16),         # 148 splits: two chunks of split weights
+    ([20000], 2, 16),         # 105 splits, 32 query columns, causal
+    ([9000, 3000], 2, 16),    # 71 and 24 splits, causal
+    ([7000] * 8, 1, 16),      # 19 splits each, just above the sliced threshold
+    ([5000] * 8, 1, 16),      # 16 splits each: one CTA per column merges the whole row
+    ([12000], 1, 128),        # CTA-pair plan, 48 splits
+])
+def test_many_splits_in_a_small_combine_grid(dev, lens, s_q, heads):
+    d = workloads.build(len(lens), s_q, heads, ("list", lens), seed=95 + len(lens) + s_q, causal=(s_q > 1))
+    print(check(d, dev, num_sms=148))
+
+
+def test_many_splits_fp32_output_explicit_combine_and_poison(dev):
+    """The sliced merge on fp32 output meets the literal RMSE; the explicit
+    combine equals the fused launch bit for bit; with NaN-filled workspace and
+    outputs every output element is still written."""
+    d = workloads.build(1, 1, 16, ("list", [66000]), seed=97)
+    o1, l1, _ = run_gpu(d, dev, num_sms=148, fp32_out=True)
+    ro, rl = ref(d)
+    m = helpers.compare(o1, l1, ro, rl)
+    assert m["rmse"] <= helpers.RMSE_BAR, m
+    o2, l2, _ = run_gpu(d, dev, num_sms=148, fp32_out=True, flags=bd.MLA_FLAG_NO_COMBINE)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    d = workloads.build(2, 2, 16, ("list", [9000, 3000]), seed=98, causal=True)
+    g = to_dev(d, dev)
+    dec = bd.MlaDecoder(2, 2, 16, g["kv_cache"].shape[0], g["block_table"].shape[1], True, 148, dev)
+    dec.workspace.view(torch.float32).fill_(float("nan"))
+    dec.out.fill_(float("nan"))
+    dec.lse.fill_(float("nan"))
+    dec.plan(g["cache_seqlens"])
+    out, lse = dec(g["q"], g["kv_cache"], g["block_table"], g["cache_seqlens"], g["softmax_scale"])
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    ro, rl = ref(d)
+    helpers.compare(out, lse, ro, rl)
+
+
 def test_one_plan_serves_repeated_calls(dev):
     """One plan serves many calls (e.g. every layer of one decode step)."""
     d = workloads.build(4, 2, 16, ("list", [9000, 70, 0, 2049]), seed=73, causal=True)
