@@ -1557,19 +1557,23 @@ constexpr int kCombineUnroll = 8;
 // larger arrays cost registers, fewer combine CTAs share an SM, and that
 // step is 4 us slower than at 4 (the 16-head workloads were unchanged).
 constexpr int kCombineFast = 4;
+#ifndef MLA_COMBINE_SLICES
+#define MLA_COMBINE_SLICES 8
+#endif
 // Many splits with few combine CTAs (a short batch over a long context: one
 // request over 148 CTAs has ~148 splits in 16 CTAs) make the per-thread chain
 // of row loads the step's tail: measured on B200 (graph-replayed, L2 flushed),
 // a bs1 x 16K step took 46.5 us against 18.5 us for its decode alone.  When
 // the combine grid (one CTA per request-group and column) is smaller than the
 // decode grid, the host launches kCombineSlices CTAs per column (grid z).
-// Above kCombineSliceMin splits, CTA z then merges d_v columns
-// [z * 128, z * 128 + 128) only: lane l owns four of them, and warp w takes
-// splits w, w + 4, ..., kCombineUnroll rows in flight.  Each thread walks a
-// quarter of the splits, on four times as many SMs.  The four warps' sums
-// meet in shared memory, in warp order.  Up to kCombineSliceMin splits, CTA 0
-// merges the whole row as above and the others leave.
-constexpr int kCombineSlices = 4;
+// Above kCombineSliceMin splits, CTA z then merges the d_v columns
+// [z * W, z * W + W) only, W = d_v / kCombineSlices: a row of W floats is
+// kLanes = W / 4 threads, so the CTA walks kCombineThreads / kLanes splits side
+// by side, each thread group taking every such split after its first, with
+// kCombineUnroll rows in flight.  The groups' sums meet in shared memory, in
+// group order.  Up to kCombineSliceMin splits, CTA 0 merges the whole row as
+// above and the others leave.
+constexpr int kCombineSlices = MLA_COMBINE_SLICES;
 constexpr int kCombineSliceMin = 16;
 
 template <int kCombineThreads, bool kMax>
@@ -1599,11 +1603,14 @@ template <int kDv, bool kSliced>
 __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const CombineParams p) {
     constexpr int kCombineThreads = kDv / 4;
     constexpr int kWarps = kCombineThreads / 32;
-    // the sliced launch only; a warp's lanes cover one slice
-    constexpr bool kCanSlice = kSliced && kDv == kCombineSlices * 32 * 4;
+    // the sliced launch only: a slice row is kLanes threads, kGroups of them per CTA
+    constexpr int kLanes = kDv / kCombineSlices / 4;
+    constexpr int kGroups = kCombineThreads / (kLanes > 0 ? kLanes : 1);
+    constexpr bool kCanSlice = kSliced && kLanes > 0 && kLanes <= 32 && kDv == kCombineSlices * kLanes * 4 &&
+                               kCombineThreads == kGroups * kLanes;
     __shared__ float red[kWarps];
     __shared__ float wts[kCombineThreads];
-    __shared__ float4 wsum[kWarps][32];
+    __shared__ float4 wsum[kGroups > 0 ? kGroups : 1][kLanes > 0 ? kLanes : 1];
     const int bg = blockIdx.x;
     const int n = blockIdx.y;
     // The grid after this one (the output projection, or the next decode) may
@@ -1700,31 +1707,31 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
                 sum += expf((i == threadIdx.x ? own : lse_of(i)) - mx);
             sum = combine_block_reduce<kCombineThreads, false>(sum, red);
             lstar = mx + logf(sum);
-            const int warp = threadIdx.x >> 5;
-            const float* rs = p.opart + (size_t)n * kDv + blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x & 31) * 4;
+            const int grp = threadIdx.x / kLanes;
+            const float* rs = p.opart + (size_t)n * kDv + blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x % kLanes) * 4;
             auto srow = [&](int i) { return *reinterpret_cast<const float4*>(rs + slot_i(i) * p.NG * kDv); };
             for (int c0 = 0; c0 < k; c0 += kCombineThreads) {
                 const int cn = k - c0 < kCombineThreads ? k - c0 : kCombineThreads;
                 __syncthreads();  // the previous chunk's weights are consumed
                 if (threadIdx.x < cn) wts[threadIdx.x] = expf((c0 == 0 ? own : lse_of(c0 + threadIdx.x)) - lstar);
                 __syncthreads();
-                int j = warp;
-                for (; j + kWarps * (kCombineUnroll - 1) < cn; j += kWarps * kCombineUnroll) {
+                int j = grp;
+                for (; j + kGroups * (kCombineUnroll - 1) < cn; j += kGroups * kCombineUnroll) {
                     float4 v[kCombineUnroll];
 #pragma unroll
-                    for (int u = 0; u < kCombineUnroll; ++u) v[u] = srow(c0 + j + kWarps * u);
+                    for (int u = 0; u < kCombineUnroll; ++u) v[u] = srow(c0 + j + kGroups * u);
 #pragma unroll
-                    for (int u = 0; u < kCombineUnroll; ++u) fma4(acc, wts[j + kWarps * u], v[u]);
+                    for (int u = 0; u < kCombineUnroll; ++u) fma4(acc, wts[j + kGroups * u], v[u]);
                 }
-                for (; j < cn; j += kWarps) fma4(acc, wts[j], srow(c0 + j));
+                for (; j < cn; j += kGroups) fma4(acc, wts[j], srow(c0 + j));
             }
         }
-        wsum[threadIdx.x >> 5][threadIdx.x & 31] = acc;
+        wsum[threadIdx.x / kLanes][threadIdx.x % kLanes] = acc;
         __syncthreads();
-        if (threadIdx.x < 32) {
+        if (threadIdx.x < kLanes) {
             acc = wsum[0][threadIdx.x];
 #pragma unroll
-            for (int w = 1; w < kWarps; ++w) {
+            for (int w = 1; w < kGroups; ++w) {
                 const float4 t = wsum[w][threadIdx.x];
                 acc.x += t.x;
                 acc.y += t.y;
@@ -1770,9 +1777,9 @@ __global__ void __launch_bounds__(kDv / 4) mla_decode_combine_kernel(const Combi
             }
         }
     }
-    const int dcol = sliced ? (int)blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x & 31) * 4 : d0;
+    const int dcol = sliced ? (int)blockIdx.z * (kDv / kCombineSlices) + (threadIdx.x % kLanes) * 4 : d0;
     const size_t o = (((size_t)b * p.s_q + s) * p.heads + head) * kDv + dcol;
-    if (!sliced || threadIdx.x < 32) {
+    if (!sliced || threadIdx.x < kLanes) {
         if (p.out_f32) {
             *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = acc;
         } else {

@@ -356,7 +356,7 @@ int launch_combine(const ColMap& cm, const Plan& pl, const void* schedule, const
     cudaLaunchConfig_t cfg = {};
     // Fewer combine CTAs than decode CTAs: several per column, so that many
     // splits are merged in d_v slices (mla_decode_combine_kernel).
-    const bool slices = kDvT == kCombineSlices * 128 && (int64_t)c.BG * pl.gr.NG < pl.ctas;
+    const bool slices = kDvT == kDv && (int64_t)c.BG * pl.gr.NG < pl.ctas;
     cfg.gridDim = dim3(c.BG, pl.gr.NG, slices ? kCombineSlices : 1);
     cfg.blockDim = dim3(kDvT / 4);
     cfg.dynamicSmemBytes = 0;
