@@ -273,7 +273,7 @@ def test_explicit_combine_matches_fused_launch(dev):
 
 
 # Short batches over long contexts: many splits per column in a small combine
-# grid, which the library merges in d_v slices (four CTAs per column).  The
+# grid, which the library merges in d_v slices (several CTAs per column).  The
 # split counts in the comments are the plan's at 148 CTAs.
 @pytest.mark.parametrize("lens,s_q,heads", [
     ([66000], 1, 16),         # 148 splits: two chunks of split weights
