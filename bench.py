@@ -559,8 +559,9 @@ def run_ours(args, w):
 
 
 def run_e2e(args, w, d, dims, kv, sched, ws, stream, dev, world):
-    """Per step: pinned host q / block_table / seqlens -> device, schedule,
-    decode, combine, out / lse -> pinned host, stream synchronised (the caller
+    """Per step: pinned host q / block_table / seqlens -> device, decode
+    (plan built in the kernel), combine, out / lse -> pinned host, stream
+    synchronised (the caller
     reads the result).  The KV cache stays resident: it is the model's state,
     not a per-step input.  The inputs travel as one packed host->device copy
     and the outputs as one packed device->host copy (the API calls take views
@@ -829,8 +830,8 @@ def run_sweep(args):
 def run_gqa_bench(args):
     """The GQLA GQA path (group-expanded cache: per token 8 groups of 128-wide
     keys and values plus a 64-wide shared RoPE key) at bs16, s_q 2 causal,
-    128 query heads, 16K context: step (schedule + decode + combine) and
-    decode kernel alone, graph-replayed; bytes = every cache row once + Q + O
+    128 query heads, 16K context: step (decode with its plan built in the
+    kernel, then the combine) and decode kernel alone, graph-replayed; bytes = every cache row once + Q + O
     + LSE, FLOPs = 2 * h_q * s_q * L * (192 + 128)."""
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
