@@ -2,7 +2,6 @@
 split-KV plan.  Test infrastructure only."""
 from __future__ import annotations
 
-import math
 import re
 import os
 

@@ -6,7 +6,6 @@ run of the exchange on the CPU, and on one GPU the CUDA merge
 The merge oracle (oracle/merge.py) is pinned here against the whole-context
 decode oracle: merging the shards' exact results must reproduce it to fp64
 rounding, with causal s_q = 2 and with ranks that hold no page of a request."""
-import ctypes
 import datetime
 import os
 

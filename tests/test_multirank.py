@@ -4,7 +4,6 @@ the slowest rank's and bytes add up; no collective touches the data path."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
